@@ -1,0 +1,779 @@
+// HSTU attention forward for B200 (sm_100a): bf16 inputs, head dim 128, fp32
+// accumulation in tensor memory.
+//
+// Computes, per user b, head h and query row i (section "HSTU" of "How
+// Generative Recommenders Are Redefining RecSys at Scale": SiLU weighting in
+// place of softmax plus a relative attention bias):
+//     O[i] = scale * sum_{j in M(i)} SiLU(q_i . k_j + rab(i, j)) v_j
+// with the causal-suffix mask (queries are the last n_q of the user's n_k
+// tokens, key j visible iff pos_j <= pos_i) or the candidate mask (candidate c
+// sees every cached token of its user plus itself).  Keys/values come either
+// from token-major jagged tensors or, page by page, from the paged KV table
+// (the attention kernel reads the cache directly: "Déploiement de
+// recommandeurs génératifs avec NVIDIA Dynamo-Triton et HSTU", section
+// "Comment cela fonctionne").
+//
+// Structure (one persistent CTA per SM, 384 threads):
+//   warp 0      TMA producer: Q tile (128 x 128), K ring (3 x 128 x 128),
+//               V ring (2 x 128 x 128), all 128-byte swizzled.  Paged keys are
+//               four 32-token page boxes per 128-key tile.
+//   warp 1      tcgen05 issuer: S = Q K^T into TMEM (two S buffers), then
+//               O += P V with P read from TMEM (two bf16 P buffers).
+//   warps 4-11  two "pointwise" warpgroups, alternating key tiles: read S
+//               from TMEM, add the bias, apply the mask, SiLU (via tanh), pack P
+//               to bf16 in TMEM; then the epilogue (O * scale -> bf16 or fp32
+//               split partial).
+// There is no softmax, so there is no running max and no rescaling of O, and
+// key splits of one query tile add exactly (the candidate path splits keys).
+// Work items (user, head, query tile, split) run longest-first: query tiles
+// are visited from the highest tile index down.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "attn.h"
+#include "sm100.cuh"
+
+namespace hstu {
+namespace {
+
+constexpr int BM = 128;            // query rows per tile
+constexpr int BN = 128;            // keys per tile
+constexpr int HD = 128;            // head dim
+constexpr int KST = 3;             // K ring depth
+constexpr int VST = 2;             // V ring depth
+constexpr int kThreads = 384;
+constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
+constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
+constexpr int kMaxUsers = 2048;
+constexpr int kMaxRab = 256;
+
+constexpr uint32_t TM_O = 0, TM_S0 = 128, TM_P0 = 384;  // S1 = S0 + 128, P1 = P0 + 64
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
+
+struct __align__(1024) Smem {
+  uint8_t q[kTileBytes];
+  uint8_t k[KST][kTileBytes];
+  uint8_t v[VST][kTileBytes];
+  int64_t kts[8][BN];          // key timestamps, one copy per pointwise warp
+  float pos_tab[kMaxRab];
+  float time_tab[kMaxRab];
+  int qt[kMaxUsers];           // query tiles per user
+  uint64_t q_full, q_empty;
+  uint64_t k_full[KST], k_empty[KST];
+  uint64_t v_full[VST], v_empty[VST];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t o_full, o_empty;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct KParams {
+  int B, H, mode, n_split, kps;
+  const int64_t* q_off;
+  const int64_t* kv_off;
+  const int64_t* users;
+  const int32_t* page_lists;
+  const int64_t* lengths;
+  int64_t max_users;
+  int max_ppu;
+  int64_t n_pages;
+  const float* pos_table;
+  int n_pos;
+  const float* time_table;
+  int n_time;
+  const int64_t* ts;
+  float scale;
+  __nv_bfloat16* out;
+  int64_t out_stride;
+  float* partial;
+  int64_t total_q;
+  int* err;
+};
+
+// ------------------------------------------------------------ scheduling
+__device__ __forceinline__ int count_users_above(const int* qt, int B, int lvl, int lane) {
+  int c = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const bool p = b < B && qt[b] > lvl;
+    c += __popc(__ballot_sync(0xffffffffu, p));
+  }
+  return c;
+}
+
+__device__ __forceinline__ int nth_user_above(const int* qt, int B, int lvl, int n, int lane) {
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const bool p = b < B && qt[b] > lvl;
+    unsigned m = __ballot_sync(0xffffffffu, p);
+    const int c = __popc(m);
+    if (n < c) {
+      for (int i = 0; i < n; ++i) m &= m - 1;
+      return b0 + __ffs(m) - 1;
+    }
+    n -= c;
+  }
+  return -1;
+}
+
+// Item order: query-tile level from the highest down; within a level, users in
+// order, then heads, then key splits.  Warp-collective (all lanes agree).
+struct Sched {
+  int lvl;
+  long long base, cnt;
+  int B, HS;
+  __device__ void init(const int* qt, int B_, int HS_, int lane) {
+    B = B_;
+    HS = HS_;
+    int mx = 0;
+    for (int b = lane; b < B; b += 32) mx = max(mx, qt[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    lvl = mx - 1;
+    base = 0;
+    cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, lane) * HS : 0;
+  }
+  __device__ bool item(long long t, const int* qt, int lane, int& b, int& m, int& rem) {
+    while (lvl >= 0 && t >= base + cnt) {
+      base += cnt;
+      --lvl;
+      cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, lane) * HS : 0;
+    }
+    if (lvl < 0) return false;
+    const long long r = t - base;
+    rem = (int)(r % HS);
+    b = nth_user_above(qt, B, lvl, (int)(r / HS), lane);
+    m = lvl;
+    return b >= 0;
+  }
+};
+
+struct Item {
+  int b, h, m, s;
+  int64_t q_row0;   // global query row of tile row 0
+  int nvalid;       // valid query rows in the tile
+  int64_t p0;       // position of query row 0
+  int64_t n_k;      // keys of the user (cached length / sequence length)
+  int64_t kv_row0;  // contiguous: global row of key position 0
+  int64_t user;     // paged: user id
+  int n_main;       // tiles from the main key source; tile n_main is the candidate tile
+  int t0, t1;       // this item's tile range
+};
+
+template <bool PAGED, bool CAND>
+__device__ __forceinline__ Item make_item(const KParams& P, int b, int m, int rem) {
+  Item it;
+  it.b = b;
+  it.m = m;
+  it.h = rem / P.n_split;
+  it.s = rem % P.n_split;
+  const int64_t qs = P.q_off[b], nq = P.q_off[b + 1] - qs;
+  it.q_row0 = qs + (int64_t)BM * m;
+  it.nvalid = (int)min64(BM, nq - (int64_t)BM * m);
+  if (PAGED) {
+    // an out-of-range user id has no cached tokens (and no page list is read)
+    const int64_t u = P.users[b];
+    const bool known = u >= 0 && u < P.max_users;
+    it.user = known ? u : 0;
+    it.n_k = known ? P.lengths[u] : 0;
+    it.kv_row0 = 0;
+  } else {
+    it.user = 0;
+    it.kv_row0 = P.kv_off[b];
+    it.n_k = P.kv_off[b + 1] - it.kv_row0;
+  }
+  int total;
+  if (CAND) {
+    it.p0 = it.n_k;
+    it.n_main = (int)((it.n_k + BN - 1) / BN);
+    total = it.n_main + 1;
+  } else {
+    it.p0 = it.n_k - nq + (int64_t)BM * m;
+    const int64_t last = it.p0 + it.nvalid - 1;
+    it.n_main = last >= 0 ? (int)(last / BN) + 1 : 0;
+    total = it.n_main;
+  }
+  if (P.n_split > 1) {
+    it.t0 = it.s * P.kps;
+    it.t1 = min(total, it.t0 + P.kps);
+  } else {
+    it.t0 = 0;
+    it.t1 = total;
+  }
+  return it;
+}
+
+__device__ __forceinline__ void record_timeout(const KParams& P, Smem& sm) {
+  atomicExch(P.err, DEV_ERR_TIMEOUT);
+  *(volatile int*)&sm.abort_flag = 1;
+}
+
+// ------------------------------------------------------------ the kernel
+template <bool PAGED, bool CAND>
+__global__ void __launch_bounds__(kThreads, 1)
+    hstu_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_kc,
+                           const __grid_constant__ CUtensorMap tm_vc, const KParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- setup
+  for (int b = tid; b < P.B; b += kThreads) {
+    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
+    sm.qt[b] = (int)((nq + BM - 1) / BM);
+  }
+  for (int i = tid; i < kMaxRab; i += kThreads) {
+    sm.pos_tab[i] = (P.pos_table && i < P.n_pos) ? P.pos_table[i] : 0.f;
+    sm.time_tab[i] = (P.time_table && i < P.n_time) ? P.time_table[i] : 0.f;
+  }
+  if (tid == 0) {
+    sm.abort_flag = 0;
+    mbar_init(smem_u32(&sm.q_full), 1);
+    mbar_init(smem_u32(&sm.q_empty), 1);
+    for (int i = 0; i < KST; ++i) {
+      mbar_init(smem_u32(&sm.k_full[i]), 1);
+      mbar_init(smem_u32(&sm.k_empty[i]), 1);
+    }
+    for (int i = 0; i < VST; ++i) {
+      mbar_init(smem_u32(&sm.v_full[i]), 1);
+      mbar_init(smem_u32(&sm.v_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.s_empty[i]), 4);
+      mbar_init(smem_u32(&sm.p_full[i]), 4);
+      mbar_init(smem_u32(&sm.p_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&sm.o_full), 1);
+    mbar_init(smem_u32(&sm.o_empty), 8);
+    mbar_init(smem_u32(&sm.mma_done), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    if (CAND) {
+      tma_prefetch_desc(&tm_kc);
+      tma_prefetch_desc(&tm_vc);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int HS = P.H * P.n_split;
+
+  if (warp == 0) {
+    // =============================================== TMA producer
+    Sched sc;
+    sc.init(sm.qt, P.B, HS, lane);
+    uint32_t kc = 0, vc = 0, qi = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x;; t += gridDim.x) {
+      int b, m, rem;
+      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (it.t0 >= it.t1) continue;
+      if (lane == 0) {
+        ok = mbar_wait(smem_u32(&sm.q_empty), (qi & 1) ^ 1);
+        if (ok) {
+          const uint32_t bar = smem_u32(&sm.q_full);
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          tma_load_3d(smem_u32(sm.q), &tm_q, bar, 0, it.h, (int)it.q_row0);
+          tma_load_3d(smem_u32(sm.q) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++qi;
+      // Issue order K0, K1, V0, K2, V1, ... keeps K one tile ahead of V.
+      const int nt = it.t1 - it.t0;
+      for (int i = 0; i <= nt && ok; ++i) {
+        if (lane == 0) {
+          for (int which = 0; which < 2 && ok; ++which) {
+            // which == 0: K of tile i ; which == 1: V of tile i-1
+            const int ti = which == 0 ? i : i - 1;
+            if (ti < 0 || ti >= nt) continue;
+            const int tile = it.t0 + ti;
+            uint32_t slot, bar, dst;
+            if (which == 0) {
+              slot = kc % KST;
+              ok = mbar_wait(smem_u32(&sm.k_empty[slot]), ((kc / KST) & 1) ^ 1);
+              bar = smem_u32(&sm.k_full[slot]);
+              dst = smem_u32(sm.k[slot]);
+              ++kc;
+            } else {
+              slot = vc % VST;
+              ok = mbar_wait(smem_u32(&sm.v_empty[slot]), ((vc / VST) & 1) ^ 1);
+              bar = smem_u32(&sm.v_full[slot]);
+              dst = smem_u32(sm.v[slot]);
+              ++vc;
+            }
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar, kTileBytes);
+            if (CAND && tile == it.n_main) {
+              const CUtensorMap* tm = which == 0 ? &tm_kc : &tm_vc;
+              tma_load_3d(dst, tm, bar, 0, it.h, (int)it.q_row0);
+              tma_load_3d(dst + kHalfBytes, tm, bar, 64, it.h, (int)it.q_row0);
+            } else if (PAGED) {
+              const int32_t* plist = P.page_lists + it.user * (int64_t)P.max_ppu;
+#pragma unroll
+              for (int pg = 0; pg < 4; ++pg) {
+                const int idx = tile * 4 + pg;
+                int64_t page = idx < P.max_ppu ? (int64_t)plist[idx] : -1;
+                if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
+                const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
+                tma_load_2d(dst + pg * 4096, &tm_k, bar, 0, row);
+                tma_load_2d(dst + kHalfBytes + pg * 4096, &tm_k, bar, 64, row);
+              }
+            } else {
+              const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
+              const int row = (int)(it.kv_row0 + (int64_t)tile * BN);
+              tma_load_3d(dst, tm, bar, 0, it.h, row);
+              tma_load_3d(dst + kHalfBytes, tm, bar, 64, it.h, row);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      record_timeout(P, sm);
+      // let copies already in flight land before the CTA can exit
+      for (uint32_t i = 0; i < KST && i < kc; ++i) {
+        const uint32_t c = kc - 1 - i;
+        mbar_wait(smem_u32(&sm.k_full[c % KST]), (c / KST) & 1);
+      }
+      for (uint32_t i = 0; i < VST && i < vc; ++i) {
+        const uint32_t c = vc - 1 - i;
+        mbar_wait(smem_u32(&sm.v_full[c % VST]), (c / VST) & 1);
+      }
+      if (qi > 0) mbar_wait(smem_u32(&sm.q_full), (qi - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // =============================================== MMA issuer
+    Sched sc;
+    sc.init(sm.qt, P.B, HS, lane);
+    uint32_t kc = 0, vc = 0, qi = 0, g = 0;
+    bool ok = true;
+    const uint32_t q_base = smem_u32(sm.q);
+    auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+      const uint32_t pb = gp & 1;
+      if (!mbar_wait(smem_u32(&sm.p_full[pb]), (gp >> 1) & 1)) return false;
+      const uint32_t slot = vc % VST;
+      if (!mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1)) return false;
+      if (first && !mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1)) return false;
+      tc_fence_after();
+      const uint32_t v_base = smem_u32(sm.v[slot]);
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key groups
+        // 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
+        const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
+        umma_ts(tmem + TM_O, tmem + TM_P0 + pb * 64 + kk * 8, bdesc, kIdescPV,
+                (first && kk == 0) ? 0u : 1u);
+      }
+      umma_commit(smem_u32(&sm.v_empty[slot]));
+      umma_commit(smem_u32(&sm.p_empty[pb]));
+      ++vc;
+      return true;
+    };
+    for (long long t = blockIdx.x; ok; t += gridDim.x) {
+      int b, m, rem;
+      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (it.t0 >= it.t1) continue;
+      if (lane == 0) {
+        ok = mbar_wait(smem_u32(&sm.q_full), qi & 1);
+        const int nt = it.t1 - it.t0;
+        for (int i = 0; i < nt && ok; ++i) {
+          const uint32_t sb = g & 1;
+          ok = mbar_wait(smem_u32(&sm.s_empty[sb]), ((g >> 1) & 1) ^ 1);
+          const uint32_t slot = kc % KST;
+          if (ok) ok = mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sm.k[slot]);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+            umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&sm.k_empty[slot]));
+          umma_commit(smem_u32(&sm.s_full[sb]));
+          ++kc;
+          if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty));
+          if (i > 0) ok = issue_pv(g - 1, i == 1);
+          ++g;
+        }
+        if (ok) ok = issue_pv(g - 1, nt == 1);
+        if (ok) umma_commit(smem_u32(&sm.o_full));
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      g = __shfl_sync(0xffffffffu, g, 0);
+      kc = __shfl_sync(0xffffffffu, kc, 0);
+      vc = __shfl_sync(0xffffffffu, vc, 0);
+      ++qi;
+    }
+    if (lane == 0) {
+      if (!ok) record_timeout(P, sm);
+      // all MMAs issued by this thread must finish before TMEM is released
+      umma_commit(smem_u32(&sm.mma_done));
+      mbar_wait(smem_u32(&sm.mma_done), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // =============================================== pointwise + epilogue
+    const int wg = (warp - 4) >> 2;                 // 0 or 1
+    const int sub = warp & 3;                       // TMEM lane quarter
+    const int r = sub * 32 + lane;                  // tile row owned by this thread
+    const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+    const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
+    Sched sc;
+    sc.init(sm.qt, P.B, HS, lane);
+    uint32_t qi = 0, g = 0;
+    bool ok = true;
+    int64_t* kts = sm.kts[warp - 4];
+    for (long long t = blockIdx.x; ok; t += gridDim.x) {
+      int b, m, rem;
+      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (it.t0 >= it.t1) continue;
+      const int64_t qp = it.p0 + r;                 // this row's query position
+      int64_t ts_q = 0;
+      if (use_time) {
+        const int64_t qpc = min64(max64(qp, 0), max64(it.n_k - 1, 0));
+        ts_q = it.n_k > 0 ? P.ts[it.kv_row0 + qpc] : 0;
+      }
+      const int n_pos_m1 = P.n_pos - 1, n_time_m1 = P.n_time - 1;
+      for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
+        if ((int)(g & 1) != wg) continue;
+        const uint32_t sb = g & 1;
+        const bool cand_tile = CAND && tile == it.n_main;
+        const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
+        // int32 tile-relative coordinates: query position minus k0, valid keys
+        const int qrel = (int)max64(min64(qp - k0, 1 << 30), -(1 << 30));
+        const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
+        if (use_time) {
+          __syncwarp();
+          for (int i = lane; i < BN; i += 32) {
+            const int64_t kp = k0 + i;
+            kts[i] = kp < it.n_k ? P.ts[it.kv_row0 + kp] : 0;
+          }
+          __syncwarp();
+        }
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[sb]), (g >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_addr + TM_S0 + sb * 128;
+        const uint32_t p_addr = tmem + lane_addr + TM_P0 + sb * 64;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sa[32], sb2[32];
+          tmem_ld32(s_addr + half * 64, sa);
+          tmem_ld32(s_addr + half * 64 + 32, sb2);
+          tmem_wait_ld();
+          reg_fence(sa);
+          reg_fence(sb2);
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+          }
+          uint32_t packed[32];
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            float pv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = half * 64 + j + e;
+              const float s = __uint_as_float(j + e < 32 ? sa[j + e] : sb2[j + e - 32]);
+              bool valid;
+              int delta;
+              if (CAND) {
+                valid = cand_tile ? (c == r) : (c < kend);
+                delta = cand_tile ? 0 : qrel - c;
+              } else {
+                valid = c <= qrel;
+                delta = qrel - c;
+              }
+              const int bk = 31 - __clz(max(delta, 0) + 1);
+              float x = s + sm.pos_tab[min(bk, n_pos_m1)];
+              if (use_time) {
+                long long dt = ts_q - kts[c];
+                dt = dt < 0 ? 0 : dt;
+                const int bt = 63 - __clzll(dt + 1);
+                x += sm.time_tab[min(bt, n_time_m1)];
+              }
+              const float hx = 0.5f * x;
+              const float y = fmaf(hx, tanh_approx(hx), hx);
+              pv[e] = valid ? y : 0.f;
+            }
+            packed[j >> 1] = pack_bf16x2(pv[0], pv[1]);
+          }
+          if (half == 0) {
+            ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          uint32_t lo[16], hi[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            lo[j] = packed[j];
+            hi[j] = packed[16 + j];
+          }
+          tmem_st16(p_addr + half * 32, lo);
+          tmem_st16(p_addr + half * 32 + 16, hi);
+        }
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
+      }
+      if (!ok) break;
+      // ---- epilogue: this warpgroup stores columns [64 wg, 64 wg + 64)
+      ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t oa[32], ob[32];
+      const uint32_t o_addr = tmem + lane_addr + TM_O + wg * 64;
+      tmem_ld32(o_addr, oa);
+      tmem_ld32(o_addr + 32, ob);
+      tmem_wait_ld();
+      reg_fence(oa);
+      reg_fence(ob);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
+      ++qi;
+      if (r < it.nvalid && it.q_row0 + r < P.total_q) {
+        const int64_t row = it.q_row0 + r;
+        if (P.partial) {
+          float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
+                       it.h * HD + wg * 64;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            reinterpret_cast<float4*>(dst)[j / 4] =
+                make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
+                            __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+            reinterpret_cast<float4*>(dst + 32)[j / 4] =
+                make_float4(__uint_as_float(ob[j]), __uint_as_float(ob[j + 1]),
+                            __uint_as_float(ob[j + 2]), __uint_as_float(ob[j + 3]));
+          }
+        } else {
+          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + wg * 64;
+          const float sc2 = P.scale;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u, w;
+            u.x = pack_bf16x2(__uint_as_float(oa[j]) * sc2, __uint_as_float(oa[j + 1]) * sc2);
+            u.y = pack_bf16x2(__uint_as_float(oa[j + 2]) * sc2, __uint_as_float(oa[j + 3]) * sc2);
+            u.z = pack_bf16x2(__uint_as_float(oa[j + 4]) * sc2, __uint_as_float(oa[j + 5]) * sc2);
+            u.w = pack_bf16x2(__uint_as_float(oa[j + 6]) * sc2, __uint_as_float(oa[j + 7]) * sc2);
+            w.x = pack_bf16x2(__uint_as_float(ob[j]) * sc2, __uint_as_float(ob[j + 1]) * sc2);
+            w.y = pack_bf16x2(__uint_as_float(ob[j + 2]) * sc2, __uint_as_float(ob[j + 3]) * sc2);
+            w.z = pack_bf16x2(__uint_as_float(ob[j + 4]) * sc2, __uint_as_float(ob[j + 5]) * sc2);
+            w.w = pack_bf16x2(__uint_as_float(ob[j + 6]) * sc2, __uint_as_float(ob[j + 7]) * sc2);
+            reinterpret_cast<uint4*>(dst)[j / 8] = u;
+            reinterpret_cast<uint4*>(dst + 32)[j / 8] = w;
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) record_timeout(P, sm);
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Deterministic reduction of the key-split partials: for each query row,
+// sum the valid splits in split order, scale, round to bf16.
+template <bool PAGED>
+__global__ void split_reduce_kernel(KParams P, int B) {
+  const int64_t row = blockIdx.x;
+  if (row >= P.total_q || row >= P.q_off[B]) return;
+  // find the user of this row
+  int lo = 0, hi = B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (P.q_off[mid] <= row) lo = mid;
+    else hi = mid;
+  }
+  const int b = lo;
+  int64_t n_k;
+  if (PAGED) {
+    const int64_t u = P.users[b];
+    n_k = (u >= 0 && u < P.max_users) ? P.lengths[u] : 0;
+  } else {
+    n_k = P.kv_off[b + 1] - P.kv_off[b];
+  }
+  const int total = (int)((n_k + BN - 1) / BN) + 1;  // candidate layout: history tiles + 1
+  const int n_valid = min(P.n_split, (total + P.kps - 1) / P.kps);
+  const int F = P.H * HD;
+  for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_valid; ++s) {
+      const float4 x = *reinterpret_cast<const float4*>(P.partial + ((int64_t)s * P.total_q + row) * F + f);
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    __nv_bfloat16* dst = P.out + row * P.out_stride + f;
+    uint2 u;
+    u.x = pack_bf16x2(acc.x * P.scale, acc.y * P.scale);
+    u.y = pack_bf16x2(acc.z * P.scale, acc.w * P.scale);
+    *reinterpret_cast<uint2*>(dst) = u;
+  }
+}
+
+size_t smem_bytes() { return sizeof(Smem) + 1024; }
+
+template <bool PAGED, bool CAND>
+cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, int grid, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, tkc, tvc;
+  const uint64_t qrows = (uint64_t)std::max<int64_t>(p.total_q, 1);
+  if (!make_tmap_3d(&tq, p.q, HD, p.H, qrows, HD * 2, (uint64_t)p.q_stride * 2, 64, BM))
+    return cudaErrorInvalidValue;
+  if (PAGED) {
+    const uint64_t rows = (uint64_t)(p.n_pages + 1) * 2 * p.H * 32;
+    if (!make_tmap_2d(&tk, p.pool, HD, rows, HD * 2, 64, 32)) return cudaErrorInvalidValue;
+    tv = tk;
+  } else {
+    const uint64_t krows = (uint64_t)std::max<int64_t>(p.total_kv, 1);
+    if (!make_tmap_3d(&tk, p.k, HD, p.H, krows, HD * 2, (uint64_t)p.k_stride * 2, 64, BN))
+      return cudaErrorInvalidValue;
+    if (!make_tmap_3d(&tv, p.v, HD, p.H, krows, HD * 2, (uint64_t)p.v_stride * 2, 64, BN))
+      return cudaErrorInvalidValue;
+  }
+  if (CAND) {
+    if (!make_tmap_3d(&tkc, p.k, HD, p.H, qrows, HD * 2, (uint64_t)p.k_stride * 2, 64, BM))
+      return cudaErrorInvalidValue;
+    if (!make_tmap_3d(&tvc, p.v, HD, p.H, qrows, HD * 2, (uint64_t)p.v_stride * 2, 64, BM))
+      return cudaErrorInvalidValue;
+  } else {
+    tkc = tq;
+    tvc = tq;
+  }
+  auto kern = hstu_attn_sm100_kernel<PAGED, CAND>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes());
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  kern<<<grid, kThreads, smem_bytes(), stream>>>(tq, tk, tv, tkc, tvc, kp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || kp.partial == nullptr) return e;
+  split_reduce_kernel<PAGED><<<(unsigned)p.total_q, 128, 0, stream>>>(kp, p.B);
+  return cudaGetLastError();
+}
+
+// Key-split plan for the candidate path: enough (user, head, split) items to
+// cover the SMs about twice.
+void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
+  *n_split = 1;
+  *kps = 1 << 30;
+  if (p.mode != 1) return;
+  const int max_tiles = (p.max_kv + BN - 1) / BN + 1;
+  const int qt = std::max(1, (p.max_q + BM - 1) / BM);
+  const long long base_items = (long long)p.B * p.H * qt;
+  if (base_items <= 0) return;
+  int want = (int)std::min<long long>(max_tiles, (2LL * num_sms + base_items - 1) / base_items);
+  if (want <= 1) return;
+  int k = (max_tiles + want - 1) / want;
+  k = std::max(k, 2);
+  *kps = k;
+  *n_split = (max_tiles + k - 1) / k;
+  if (*n_split <= 1) {
+    *n_split = 1;
+    *kps = 1 << 30;
+  }
+}
+
+}  // namespace
+
+size_t attn_sm100_workspace_bytes(const AttnProblem& p, int num_sms) {
+  int ns, kps;
+  split_plan(p, num_sms, &ns, &kps);
+  if (ns <= 1) return 0;
+  return (size_t)ns * (size_t)p.total_q * p.H * HD * sizeof(float);
+}
+
+cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_bytes,
+                              int* err_word, cudaStream_t stream) {
+  if (p.d != HD || p.f32) return cudaErrorInvalidValue;
+  if (p.B > kMaxUsers) return cudaErrorInvalidValue;
+  if (p.B == 0 || p.total_q == 0) return cudaSuccess;
+  const int num_sms = device_sm_count();
+  KParams kp;
+  std::memset(&kp, 0, sizeof(kp));
+  kp.B = p.B;
+  kp.H = p.H;
+  kp.mode = p.mode;
+  split_plan(p, num_sms, &kp.n_split, &kp.kps);
+  kp.q_off = p.q_off;
+  kp.kv_off = p.kv_off;
+  kp.users = p.users;
+  kp.page_lists = p.page_lists;
+  kp.lengths = p.lengths;
+  kp.max_users = p.max_users;
+  kp.max_ppu = p.max_ppu;
+  kp.n_pages = p.n_pages;
+  kp.pos_table = p.pos_table;
+  kp.n_pos = p.pos_table ? p.n_pos : 1;
+  kp.time_table = p.time_table;
+  kp.n_time = p.time_table ? p.n_time : 1;
+  kp.ts = p.ts;
+  kp.scale = p.scale;
+  kp.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  kp.out_stride = p.out_stride;
+  kp.total_q = p.total_q;
+  kp.err = err_word;
+  if (kp.n_split > 1) {
+    const size_t need = attn_sm100_workspace_bytes(p, num_sms);
+    if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
+    kp.partial = reinterpret_cast<float*>(workspace);
+  }
+  const int qt = (p.max_q + BM - 1) / BM;
+  const long long items = (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
+  const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
+  if (p.paged) {
+    return p.mode == 1 ? launch_impl<true, true>(p, kp, grid, stream)
+                       : launch_impl<true, false>(p, kp, grid, stream);
+  }
+  return p.mode == 1 ? launch_impl<false, true>(p, kp, grid, stream)
+                     : launch_impl<false, false>(p, kp, grid, stream);
+}
+
+}  // namespace hstu

@@ -1,0 +1,311 @@
+// Paged GPU KV data table: allocation, append and lookup ("NVIDIA Dynamo-Triton
+// Gets End-to-End HSTU Generative Recommender Workflow", section "What the
+// workflow combines": the GPU cache is a paged KV data table with lookup,
+// allocation, append and eviction).
+//
+// Storage (all device memory, allocated once by hstu_kv_table_create):
+//   pool        [(n_pages + 1)][2 (K,V)][H][32 slots][d]; page n_pages stays
+//               zero and stands in for missing pages inside the attention
+//               kernel's tile loads
+//   free_stack  [n_pages] int32, free_top = number of free pages; the top of
+//               the stack is free_stack[free_top - 1]
+//   page_lists  [max_users][max_ppu] int32 (-1 = none), n_held [max_users]
+//   lengths     [max_users] int64 cached tokens
+//   epoch       [max_users] int32: last alloc call that listed the user
+//               (duplicate detection without clearing)
+//   done        [max_users] int32: append chunk counters (always back to 0)
+//   status      first device-side error since the last status read
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <vector>
+
+#include "kv_table.h"
+
+namespace hstu {
+
+namespace {
+
+__device__ __forceinline__ void set_status(int32_t* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+constexpr int kAllocThreads = 1024;
+
+// One CTA.  Phase 1: per-user demand and validation.  Phase 2: block-wide
+// exclusive scan of the demand in the order users are listed.  Phase 3: pop
+// pages from the top of the free stack (user 0 first).
+__global__ void __launch_bounds__(kAllocThreads)
+    kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new, int B,
+                    int32_t* page_ids_out, int page_ids_cap, int32_t epoch) {
+  __shared__ int64_t s_chunk[kAllocThreads];
+  __shared__ int s_bad;
+  __shared__ int64_t s_total;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  const int per = (B + kAllocThreads - 1) / kAllocThreads;
+  const int b0 = tid * per, b1 = min(B, b0 + per);
+  // phase 1
+  int64_t mysum = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int64_t u = users[b], n = n_new[b];
+    if (u < 0 || u >= t.max_users || n < 0) {
+      atomicOr(&s_bad, 1);
+      continue;
+    }
+    if (atomicExch(&t.epoch[u], epoch) == epoch) atomicOr(&s_bad, 1);  // listed twice
+    const int64_t want = (t.lengths[u] + n + t.page_size - 1) / t.page_size;
+    int64_t need = want - t.n_held[u];
+    need = need < 0 ? 0 : need;
+    if (t.n_held[u] + need > t.max_ppu) atomicOr(&s_bad, 1);
+    mysum += need;
+  }
+  s_chunk[tid] = mysum;
+  __syncthreads();
+  // phase 2: inclusive scan of the per-thread sums (Hillis-Steele)
+  for (int off = 1; off < kAllocThreads; off <<= 1) {
+    const int64_t x = tid >= off ? s_chunk[tid - off] : 0;
+    __syncthreads();
+    s_chunk[tid] += x;
+    __syncthreads();
+  }
+  if (tid == kAllocThreads - 1) s_total = s_chunk[tid];
+  __syncthreads();
+  const int64_t total = s_total;
+  const int64_t top = *t.free_top;
+  if (s_bad) {
+    if (tid == 0) set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
+    return;
+  }
+  if (total > top) {
+    if (tid == 0) set_status(t.status, 2 /* HSTU_ERR_OUT_OF_PAGES */);
+    return;
+  }
+  // phase 3
+  int64_t pre = s_chunk[tid] - mysum;  // exclusive prefix of this thread's first user
+  for (int b = b0; b < b1; ++b) {
+    const int64_t u = users[b];
+    const int64_t want = (t.lengths[u] + n_new[b] + t.page_size - 1) / t.page_size;
+    int64_t need = want - t.n_held[u];
+    need = need < 0 ? 0 : need;
+    const int held = t.n_held[u];
+    for (int64_t k = 0; k < need; ++k) {
+      const int32_t pid = t.free_stack[top - 1 - (pre + k)];
+      t.page_lists[u * (int64_t)t.max_ppu + held + k] = pid;
+      if (page_ids_out && pre + k < page_ids_cap) page_ids_out[pre + k] = pid;
+    }
+    t.n_held[u] = held + (int)need;
+    pre += need;
+  }
+  if (page_ids_out)
+    for (int64_t i = total + tid; i < page_ids_cap; i += kAllocThreads) page_ids_out[i] = -1;
+  __syncthreads();
+  if (tid == 0) *t.free_top = (int32_t)(top - total);
+}
+
+constexpr int kAppendTok = 8;   // tokens per CTA
+constexpr int kCopyThreads = 256;
+
+// grid (chunks, B): CTA (c, b) copies tokens [c*kAppendTok, ...) of user b.
+// The length is read before any copy and advanced by the last CTA of the user.
+template <int ESZ>
+__global__ void __launch_bounds__(kCopyThreads)
+    kv_append_kernel(KvTableDev t, const int64_t* users, const uint8_t* k_new, const uint8_t* v_new,
+                     const int64_t* new_offsets) {
+  const int b = blockIdx.y;
+  const int64_t u = users[b];
+  const int64_t s = new_offsets[b], n = new_offsets[b + 1] - s;
+  const int n_chunks = (int)((n + kAppendTok - 1) / kAppendTok);
+  if (blockIdx.x >= n_chunks) return;
+  if (u < 0 || u >= t.max_users) {
+    if (threadIdx.x == 0) set_status(t.status, 1);
+    return;
+  }
+  const int64_t len = t.lengths[u];
+  const bool fits = len + n <= (int64_t)t.n_held[u] * t.page_size;
+  if (fits) {
+    const int row_vec = t.H * t.d * ESZ / 16;     // 16-byte vectors per token row
+    const int vec_per_head = t.d * ESZ / 16;
+    const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
+    const int ntok = (int)((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok);
+    for (int i = threadIdx.x; i < ntok * row_vec * 2; i += kCopyThreads) {
+      const int kv = i / (ntok * row_vec);
+      const int rem = i % (ntok * row_vec);
+      const int tk = rem / row_vec, v = rem % row_vec;
+      const int h = v / vec_per_head, e16 = v % vec_per_head;
+      const int64_t src_row = s + tok0 + tk;
+      const int64_t pos = len + tok0 + tk;
+      const int32_t page = t.page_lists[u * (int64_t)t.max_ppu + pos / t.page_size];
+      const int slot = (int)(pos % t.page_size);
+      const uint8_t* src = (kv ? v_new : k_new) + src_row * (int64_t)t.H * t.d * ESZ;
+      const uint4 x = reinterpret_cast<const uint4*>(src)[v];
+      uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
+                     ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
+      reinterpret_cast<uint4*>(dst)[e16] = x;
+    }
+  } else if (threadIdx.x == 0 && blockIdx.x == 0) {
+    set_status(t.status, 1);
+  }
+  // the last CTA of this user commits the new length
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int prev = atomicAdd(&t.done[u], 1);
+    if (prev == n_chunks - 1) {
+      if (fits) t.lengths[u] = len + n;
+      t.done[u] = 0;
+      __threadfence();
+    }
+  }
+}
+
+// grid (chunks, B).  Chunk 0 also writes the length and the page table row.
+template <int ESZ>
+__global__ void __launch_bounds__(kCopyThreads)
+    kv_lookup_kernel(KvTableDev t, const int64_t* users, int64_t* cached_len_out,
+                     int32_t* page_table_out, int max_pages, uint8_t* k_out, uint8_t* v_out,
+                     const int64_t* out_offsets) {
+  const int b = blockIdx.y;
+  const int64_t u = users[b];
+  const bool valid_user = u >= 0 && u < t.max_users;
+  const int64_t len = valid_user ? t.lengths[u] : 0;
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0) {
+      if (cached_len_out) cached_len_out[b] = len;
+      if (!valid_user) set_status(t.status, 1);
+    }
+    if (page_table_out) {
+      const int held = valid_user ? t.n_held[u] : 0;
+      for (int p = threadIdx.x; p < max_pages; p += kCopyThreads)
+        page_table_out[(int64_t)b * max_pages + p] =
+            p < held ? t.page_lists[u * (int64_t)t.max_ppu + p] : -1;
+    }
+  }
+  if (!k_out || !valid_user) return;
+  const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
+  if (tok0 >= len) return;
+  const int ntok = (int)((len - tok0) < kAppendTok ? (len - tok0) : kAppendTok);
+  const int row_vec = t.H * t.d * ESZ / 16;
+  const int vec_per_head = t.d * ESZ / 16;
+  const int64_t o = out_offsets[b];
+  for (int i = threadIdx.x; i < ntok * row_vec * 2; i += kCopyThreads) {
+    const int kv = i / (ntok * row_vec);
+    const int rem = i % (ntok * row_vec);
+    const int tk = rem / row_vec, v = rem % row_vec;
+    const int h = v / vec_per_head, e16 = v % vec_per_head;
+    const int64_t pos = tok0 + tk;
+    const int32_t page = t.page_lists[u * (int64_t)t.max_ppu + pos / t.page_size];
+    const int slot = (int)(pos % t.page_size);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(t.pool) +
+                         ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
+    uint8_t* dst = (kv ? v_out : k_out) + (o + pos) * (int64_t)t.H * t.d * ESZ;
+    reinterpret_cast<uint4*>(dst)[v] = reinterpret_cast<const uint4*>(src)[e16];
+  }
+}
+
+}  // namespace
+
+cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order) {
+  const size_t page_bytes = (size_t)2 * t->H * t->page_size * t->d * t->esize;
+  cudaError_t e;
+  e = cudaMalloc(&t->pool, page_bytes * (size_t)(t->n_pages + 1));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->pool, 0, page_bytes * (size_t)(t->n_pages + 1));
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->free_stack, sizeof(int32_t) * (size_t)std::max<int64_t>(t->n_pages, 1));
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->free_top, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->page_lists, sizeof(int32_t) * (size_t)t->max_users * t->max_ppu);
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->page_lists, 0xff, sizeof(int32_t) * (size_t)t->max_users * t->max_ppu);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->n_held, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->n_held, 0, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->lengths, sizeof(int64_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->lengths, 0, sizeof(int64_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->epoch, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->epoch, 0, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->done, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->done, 0, sizeof(int32_t) * (size_t)t->max_users);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->status, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->status, 0, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  std::vector<int32_t> order((size_t)t->n_pages);
+  for (int64_t i = 0; i < t->n_pages; ++i) order[i] = host_free_order ? host_free_order[i] : (int32_t)i;
+  if (t->n_pages > 0) {
+    e = cudaMemcpy(t->free_stack, order.data(), sizeof(int32_t) * order.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return e;
+  }
+  const int32_t top = (int32_t)t->n_pages;
+  e = cudaMemcpy(t->free_top, &top, sizeof(int32_t), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return e;
+  return cudaDeviceSynchronize();
+}
+
+void kv_table_free_storage(KvTableDev* t) {
+  cudaFree(t->pool);
+  cudaFree(t->free_stack);
+  cudaFree(t->free_top);
+  cudaFree(t->page_lists);
+  cudaFree(t->n_held);
+  cudaFree(t->lengths);
+  cudaFree(t->epoch);
+  cudaFree(t->done);
+  cudaFree(t->status);
+}
+
+cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
+                            int32_t* page_ids_out, int page_ids_cap, int32_t epoch,
+                            cudaStream_t stream) {
+  if (B == 0 && page_ids_out == nullptr) return cudaSuccess;
+  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, B, page_ids_out, page_ids_cap,
+                                                   epoch);
+  return cudaGetLastError();
+}
+
+cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
+                             const void* v_new, const int64_t* new_offsets, int B, int max_new,
+                             cudaStream_t stream) {
+  if (B == 0 || max_new <= 0) return cudaSuccess;
+  dim3 grid((max_new + kAppendTok - 1) / kAppendTok, B);
+  if (t.esize == 2)
+    kv_append_kernel<2><<<grid, kCopyThreads, 0, stream>>>(
+        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets);
+  else
+    kv_append_kernel<4><<<grid, kCopyThreads, 0, stream>>>(
+        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
+                             int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
+                             void* k_out, void* v_out, const int64_t* out_offsets, int max_len,
+                             cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  const int chunks = k_out ? std::max(1, (max_len + kAppendTok - 1) / kAppendTok) : 1;
+  dim3 grid(chunks, B);
+  if (t.esize == 2)
+    kv_lookup_kernel<2><<<grid, kCopyThreads, 0, stream>>>(
+        t, users, cached_len_out, page_table_out, max_pages, (uint8_t*)k_out, (uint8_t*)v_out,
+        out_offsets);
+  else
+    kv_lookup_kernel<4><<<grid, kCopyThreads, 0, stream>>>(
+        t, users, cached_len_out, page_table_out, max_pages, (uint8_t*)k_out, (uint8_t*)v_out,
+        out_offsets);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

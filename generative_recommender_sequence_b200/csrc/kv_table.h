@@ -1,0 +1,39 @@
+// Internal interface of the paged KV table kernels (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace hstu {
+
+// Plain-old-data view of the table's device storage, passed to kernels by value.
+struct KvTableDev {
+  int64_t n_pages;
+  int page_size, H, d, esize;
+  int64_t max_users;
+  int max_ppu;
+  void* pool;
+  int32_t* free_stack;
+  int32_t* free_top;
+  int32_t* page_lists;
+  int32_t* n_held;
+  int64_t* lengths;
+  int32_t* epoch;
+  int32_t* done;
+  int32_t* status;
+};
+
+cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order);
+void kv_table_free_storage(KvTableDev* t);
+cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
+                            int32_t* page_ids_out, int page_ids_cap, int32_t epoch,
+                            cudaStream_t stream);
+cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
+                             const void* v_new, const int64_t* new_offsets, int B, int max_new,
+                             cudaStream_t stream);
+cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
+                             int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
+                             void* k_out, void* v_out, const int64_t* out_offsets, int max_len,
+                             cudaStream_t stream);
+
+}  // namespace hstu

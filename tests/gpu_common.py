@@ -1,0 +1,67 @@
+"""Shared helpers for the GPU parity tests (tolerances from the build's contract)."""
+
+import numpy as np
+import torch
+
+import workloads
+
+BF16_MAX_ABS = 1e-2
+BF16_REL_L2 = 5e-3
+F32_REL = 1e-5
+
+
+def dev(x, dtype=None):
+    t = torch.as_tensor(np.ascontiguousarray(x))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def storage(x, dtype: str):
+    return workloads.to_torch(x, dtype).cuda()
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    diff = got - ref
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)) if diff.size else 0.0
+    max_rel = max_abs / max(float(np.max(np.abs(ref))), 1e-300) if diff.size else 0.0
+    return max_abs, rel_l2, max_rel
+
+
+def assert_bf16_close(got, ref, what=""):
+    max_abs, rel_l2, _ = errors(got, ref)
+    assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), what
+    assert max_abs <= BF16_MAX_ABS and rel_l2 <= BF16_REL_L2, \
+        f"{what}: max_abs={max_abs:.3e} rel_l2={rel_l2:.3e}"
+    return max_abs, rel_l2
+
+
+def assert_f32_close(got, ref, what=""):
+    _, rel_l2, max_rel = errors(got, ref)
+    assert rel_l2 <= F32_REL and max_rel <= F32_REL, f"{what}: rel_l2={rel_l2:.3e} max_rel={max_rel:.3e}"
+    return rel_l2, max_rel
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def sample_rows(offsets, n_random, seed=0):
+    """Rows to check at full size: first/last rows of every user and every 128-row tile
+    boundary, plus random rows."""
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(len(offsets) - 1):
+        s, e = int(offsets[b]), int(offsets[b + 1])
+        if e <= s:
+            continue
+        rows.update([s, e - 1])
+        for t in range(s, e, 128):
+            rows.update([t, min(t + 127, e - 1)])
+    T = int(offsets[-1])
+    if T:
+        rows.update(rng.integers(0, T, size=n_random).tolist())
+    return np.array(sorted(rows), dtype=np.int64)

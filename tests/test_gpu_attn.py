@@ -1,0 +1,121 @@
+"""hstu_attn_fwd on the GPU vs the fp64 oracle (jagged causal attention)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_common import (assert_bf16_close, assert_f32_close, dev, sample_rows, storage,
+                              to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    import generative_recommender_sequence_b200 as hstu
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for -m gpu tests")
+    hstu.device_check()
+
+
+def run_case(case, rows=None, stream=None):
+    import generative_recommender_sequence_b200 as hstu
+    q, k, v = (storage(x, case.dtype) for x in (case.q, case.k, case.v))
+    off = dev(case.seq_offsets)
+    pt = dev(case.pos_table)
+    tt = dev(case.time_table) if case.time_table is not None else None
+    ts = dev(case.timestamps) if case.timestamps is not None else None
+    out = hstu.attn_fwd(q, k, v, off, case.max_len, pos_table=pt, time_table=tt, timestamps=ts,
+                        scale=case.scale)
+    torch.cuda.synchronize()
+    assert hstu.last_device_error() == 0
+    got = to_np(out)
+    ref = oracle.attn_causal(case.q, case.k, case.v, case.seq_offsets, timestamps=case.timestamps,
+                             pos_table=case.pos_table, time_table=case.time_table, scale=case.scale,
+                             rows=rows)
+    return (got if rows is None else got[rows]), ref
+
+
+def test_tiny_fp32_workload():
+    case = workloads.tiny_fp32()
+    got, ref = run_case(case)
+    assert_f32_close(got, ref, "tiny fp32")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_fp32_head_dims(d):
+    case = workloads.jagged_case(50 + d, [1, 70, 129, 5], H=3, d=d, dtype="f32", n_pos=16, n_time=8)
+    got, ref = run_case(case)
+    assert_f32_close(got, ref, f"fp32 d={d}")
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_bf16_simt_head_dims(d):
+    case = workloads.jagged_case(60 + d, [3, 100, 257], H=2, d=d, dtype="bf16", n_pos=32, n_time=16)
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, f"bf16 simt d={d}")
+
+
+@pytest.mark.parametrize("lengths", [
+    [130, 300, 517],            # several tiles, ragged tails
+    [1, 128, 129, 255, 256],    # tile-boundary edge cases
+    [0, 7, 0, 384, 0],          # empty users
+    [1000],
+])
+def test_bf16_tcgen05_pos_rab(lengths):
+    case = workloads.jagged_case(7, lengths, H=4, d=128, dtype="bf16", n_pos=16)
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, f"bf16 {lengths}")
+
+
+def test_bf16_tcgen05_pos_time_rab():
+    case = workloads.jagged_case(8, [200, 640, 37, 1100], H=4, d=128, dtype="bf16", n_pos=128,
+                                 n_time=64)
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, "pos+time rab")
+
+
+def test_bf16_no_rab_and_single_head():
+    import generative_recommender_sequence_b200 as hstu
+    case = workloads.jagged_case(9, [300, 45], H=1, d=128, dtype="bf16", n_pos=16)
+    q, k, v = (storage(x, "bf16") for x in (case.q, case.k, case.v))
+    out = hstu.attn_fwd(q, k, v, dev(case.seq_offsets), case.max_len, scale=case.scale)
+    ref = oracle.attn_causal(case.q, case.k, case.v, case.seq_offsets, scale=case.scale)
+    assert_bf16_close(to_np(out), ref, "no rab")
+
+
+def test_jagged_bf16_workload_full_size_sampled():
+    """The 8-user, L~U[256,2048] workload at full size; oracle on sampled rows."""
+    case = workloads.jagged_bf16()
+    rows = sample_rows(case.seq_offsets, 1500)
+    got, ref = run_case(case, rows=rows)
+    assert_bf16_close(got, ref, "jagged_bf16 workload")
+
+
+def test_causality_and_determinism_on_gpu():
+    import generative_recommender_sequence_b200 as hstu
+    case = workloads.jagged_case(10, [600, 300], H=4, d=128, dtype="bf16", n_pos=16)
+    q, k, v = (storage(x, "bf16") for x in (case.q, case.k, case.v))
+    off, pt = dev(case.seq_offsets), dev(case.pos_table)
+    a = hstu.attn_fwd(q, k, v, off, 600, pos_table=pt, scale=case.scale).clone()
+    b = hstu.attn_fwd(q, k, v, off, 600, pos_table=pt, scale=case.scale).clone()
+    assert torch.equal(a, b)
+    i = 250
+    k2, v2 = k.clone(), v.clone()
+    k2[i + 1:600] = -k2[i + 1:600]
+    v2[i + 1:600] += 1
+    c = hstu.attn_fwd(q, k2, v2, off, 600, pos_table=pt, scale=case.scale)
+    assert torch.equal(a[: i + 1], c[: i + 1])
+    assert torch.equal(a[600:], c[600:])   # the other user is untouched
+
+
+def test_k_zero_rab_zero_gives_zero_on_gpu():
+    import generative_recommender_sequence_b200 as hstu
+    case = workloads.jagged_case(11, [333], H=2, d=128, dtype="bf16", n_pos=16)
+    q, v = storage(case.q, "bf16"), storage(case.v, "bf16")
+    k = torch.zeros_like(q)
+    out = hstu.attn_fwd(q, k, v, dev(case.seq_offsets), 333, pos_table=torch.zeros(16, device="cuda"),
+                        scale=case.scale)
+    assert torch.count_nonzero(out) == 0
