@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(NT)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = rg * 8 + i;
-      const int64_t qp = p0 + r;
+      const int64_t qp = cand ? p0 : p0 + r;   // candidates share one position
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c = kg * 4 + j;

@@ -459,7 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
       if (it.t0 >= it.t1) continue;
-      const int64_t qp = it.p0 + r;                 // this row's query position
+      // this row's query position (every candidate sits at the cached length)
+      const int64_t qp = CAND ? it.p0 : it.p0 + r;
       int64_t ts_q = 0;
       if (use_time) {
         const int64_t qpc = min64(max64(qp, 0), max64(it.n_k - 1, 0));

@@ -1,9 +1,362 @@
-// HSTU block stack (placeholder until the GEMM kernels land).
+// HSTU block stack on B200 ("How Generative Recommenders Are Redefining RecSys
+// at Scale", section "HSTU": pointwise projection, SiLU attention with a
+// relative bias, elementwise gating before the output projection):
+//
+//   per layer:  UVQK = SiLU(X W1)                  tcgen05 GEMM, SiLU epilogue
+//               A    = HSTU attention(Q, K, V)     attn_sm100 (reads UVQK in place)
+//               G    = LayerNorm(A) * U            one warp per token
+//               X    = X + G W2                    tcgen05 GEMM, residual epilogue
+//
+// bf16 storage, fp32 accumulation; UVQK, A, G and X are the bf16 tensors the
+// stack materialises.
+//
+// GEMM kernel: persistent, one CTA per SM, 192 threads.  Warp 0 issues TMA
+// (A tile 128 x 64 K-major, B tile 64 x 256 MN-major, 128-byte swizzle, 4
+// stages), warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two
+// TMEM accumulators (2 x 256 columns), warps 2-5 drain the other accumulator
+// (tcgen05.ld -> epilogue -> global) so the epilogue of tile i overlaps the
+// main loop of tile i+1.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "attn.h"
 #include "block.h"
+#include "sm100.cuh"
 
 namespace hstu {
-size_t block_workspace_bytes(int64_t, int, int, int) { return 0; }
-cudaError_t block_fwd_launch(const BlockProblem&, void*, size_t, int*, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int GBM = 128, GBN = 256, GBK = 64;
+constexpr int GST = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kABytes = GBM * GBK * 2;       // 16 KiB
+constexpr int kBBytes = GBK * GBN * 2;       // 32 KiB
+constexpr int kBBoxBytes = GBK * 64 * 2;     // one 64-column B box: 8 KiB
+constexpr uint32_t kIdescGemm = idesc_bf16_f32(GBM, GBN, true);
+
+enum { EPI_SILU = 0, EPI_RESIDUAL = 1 };
+
+struct __align__(1024) GemmSmem {
+  uint8_t a[GST][kABytes];
+  uint8_t b[GST][kBBytes];
+  uint64_t full[GST], empty[GST];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+struct GemmParams {
+  int M, N, K;
+  __nv_bfloat16* out;        // [M, N] row stride ldo
+  int64_t ldo;
+  int* err;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b, const GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (P.M + GBM - 1) / GBM, n_tiles = P.N / GBN;
+  const int tiles = m_tiles * n_tiles;
+  const int kblocks = P.K / GBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GST; ++i) {
+      mbar_init(smem_u32(&sm.full[i]), 1);
+      mbar_init(smem_u32(&sm.empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.acc_full[i]), 1);
+      mbar_init(smem_u32(&sm.acc_empty[i]), 4);
+    }
+    mbar_init(smem_u32(&sm.mma_done), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t c = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int mt = t / n_tiles, nt = t % n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb, ++c) {
+          const uint32_t s = c % GST;
+          if (!(ok = mbar_wait(smem_u32(&sm.empty[s]), ((c / GST) & 1) ^ 1))) break;
+          const uint32_t bar = smem_u32(&sm.full[s]);
+          mbar_arrive_expect_tx(bar, kABytes + kBBytes);
+          tma_load_2d(smem_u32(sm.a[s]), &tm_a, bar, kb * GBK, mt * GBM);
+#pragma unroll
+          for (int j = 0; j < GBN / 64; ++j)
+            tma_load_2d(smem_u32(sm.b[s]) + j * kBBoxBytes, &tm_b, bar, nt * GBN + j * 64, kb * GBK);
+        }
+      }
+      if (!ok) {
+        atomicExch(P.err, DEV_ERR_TIMEOUT);
+        for (uint32_t i = 0; i < GST && i < c; ++i) {
+          const uint32_t cc = c - 1 - i;
+          mbar_wait(smem_u32(&sm.full[cc % GST]), (cc / GST) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t c = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
+        const uint32_t ab = tcount & 1;
+        if (!(ok = mbar_wait(smem_u32(&sm.acc_empty[ab]), ((tcount >> 1) & 1) ^ 1))) break;
+        tc_fence_after();
+        for (int kb = 0; kb < kblocks; ++kb, ++c) {
+          const uint32_t s = c % GST;
+          if (!(ok = mbar_wait(smem_u32(&sm.full[s]), (c / GST) & 1))) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+          for (int kk = 0; kk < GBK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            // B is MN-major: 64-column boxes 8 KiB apart (LBO), 8-row k groups 1 KiB
+            // apart (SBO), 16 k-rows = 2 KiB per k-step
+            const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, kBBoxBytes, 1024);
+            umma_ss(tmem + ab * GBN, adesc, bdesc, kIdescGemm, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&sm.empty[s]));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&sm.acc_full[ab]));
+      }
+      if (!ok) atomicExch(P.err, DEV_ERR_TIMEOUT);
+      umma_commit(smem_u32(&sm.mma_done));
+      mbar_wait(smem_u32(&sm.mma_done), 0);
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+    uint32_t tcount = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
+      const int mt = t / n_tiles, nt = t % n_tiles;
+      const uint32_t ab = tcount & 1;
+      if (!mbar_wait_warp(smem_u32(&sm.acc_full[ab]), (tcount >> 1) & 1)) {
+        if (lane == 0) atomicExch(P.err, DEV_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = (int64_t)mt * GBM + r;
+      const bool valid = row < P.M;
+      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN;
+#pragma unroll 1
+      for (int ch = 0; ch < GBN / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + ab * GBN + ch * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        if (ch == GBN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.acc_empty[ab]));
+        }
+        if (!valid) continue;
+        float x[32];
+        if (EPI == EPI_SILU) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = __uint_as_float(v[j]);
+            const float h = 0.5f * a;
+            x[j] = fmaf(h, tanh_approx(h), h);
+          }
+        } else {
+          const uint4* res = reinterpret_cast<const uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = res[q];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+              x[q * 8 + 2 * e] = __uint_as_float(v[q * 8 + 2 * e]) + __bfloat162float(p.x);
+              x[q * 8 + 2 * e + 1] = __uint_as_float(v[q * 8 + 2 * e + 1]) + __bfloat162float(p.y);
+            }
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 u;
+          u.x = pack_bf16x2(x[q * 8 + 0], x[q * 8 + 1]);
+          u.y = pack_bf16x2(x[q * 8 + 2], x[q * 8 + 3]);
+          u.z = pack_bf16x2(x[q * 8 + 4], x[q * 8 + 5]);
+          u.w = pack_bf16x2(x[q * 8 + 6], x[q * 8 + 7]);
+          dst[q] = u;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
+
+// G[t, :] = LayerNorm(A[t, :]) * U[t, :] over F = 512 features; one warp per
+// token, 16 features per lane, two-pass mean / biased variance in fp32.
+__global__ void __launch_bounds__(256)
+    ln_gate_kernel(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ u,
+                   int64_t ldu, __nv_bfloat16* __restrict__ g, int64_t T, float eps) {
+  constexpr int F = 512;
+  const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const uint4* ar = reinterpret_cast<const uint4*>(a + t * F) + lane * 2;
+  const uint4* ur = reinterpret_cast<const uint4*>(u + t * ldu) + lane * 2;
+  float x[16], w[16];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint4 av = ar[q], uv = ur[q];
+    const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 pa = *reinterpret_cast<const __nv_bfloat162*>(&aw[e]);
+      const __nv_bfloat162 pu = *reinterpret_cast<const __nv_bfloat162*>(&uw[e]);
+      x[q * 8 + 2 * e] = __bfloat162float(pa.x);
+      x[q * 8 + 2 * e + 1] = __bfloat162float(pa.y);
+      w[q * 8 + 2 * e] = __bfloat162float(pu.x);
+      w[q * 8 + 2 * e + 1] = __bfloat162float(pu.y);
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) s += x[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s * (1.f / F);
+  float v = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v = fmaf(x[i] - mean, x[i] - mean, v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const float inv = rsqrtf(v * (1.f / F) + eps);
+  uint4* gr = reinterpret_cast<uint4*>(g + t * F) + lane * 2;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    uint4 o;
+    o.x = pack_bf16x2((x[q * 8 + 0] - mean) * inv * w[q * 8 + 0], (x[q * 8 + 1] - mean) * inv * w[q * 8 + 1]);
+    o.y = pack_bf16x2((x[q * 8 + 2] - mean) * inv * w[q * 8 + 2], (x[q * 8 + 3] - mean) * inv * w[q * 8 + 3]);
+    o.z = pack_bf16x2((x[q * 8 + 4] - mean) * inv * w[q * 8 + 4], (x[q * 8 + 5] - mean) * inv * w[q * 8 + 5]);
+    o.w = pack_bf16x2((x[q * 8 + 6] - mean) * inv * w[q * 8 + 6], (x[q * 8 + 7] - mean) * inv * w[q * 8 + 7]);
+    gr[q] = o;
+  }
+}
+
+size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
+
+// out[M, N] (ld ldo) = epi(A[M, K] (ld lda) @ B[K, N] (ld ldb)); residual
+// epilogue reads out before writing it.
+template <int EPI>
+cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb, void* out,
+                        int64_t ldo, int M, int N, int K, int* err, cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  if (N % GBN != 0 || K % GBK != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, GBK, GBM))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, Bw, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 2, 64, GBK))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_bf16_kernel<EPI>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm_smem_bytes());
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int tiles = ((M + GBM - 1) / GBM) * (N / GBN);
+  const int grid = std::max(1, std::min(tiles, device_sm_count()));
+  GemmParams p{M, N, K, reinterpret_cast<__nv_bfloat16*>(out), ldo, err};
+  kern<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+size_t block_workspace_bytes(int64_t T, int d_model, int H, int dh) {
+  const size_t F = (size_t)H * dh;
+  return align256((size_t)T * 4 * F * 2) + align256((size_t)T * F * 2) * 2;
+}
+
+cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_bytes, int* err_word,
+                             cudaStream_t stream) {
+  const int F = p.H * p.dh;
+  if (p.dh != 128 || F != p.d_model || F != 512) return cudaErrorNotSupported;
+  if (ws_bytes < block_workspace_bytes(p.T, p.d_model, p.H, p.dh)) return cudaErrorInvalidValue;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* uvqk = reinterpret_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)p.T * 4 * F * 2));
+  __nv_bfloat16* gate =
+      reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)p.T * 4 * F * 2) + align256((size_t)p.T * F * 2));
+  const int M = (int)p.T;
+  for (int l = 0; l < p.n_layers; ++l) {
+    cudaError_t e = gemm_launch<EPI_SILU>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+                                          p.d_model, err_word, stream);
+    if (e != cudaSuccess) return e;
+    AttnProblem a;
+    a.B = p.B;
+    a.H = p.H;
+    a.d = p.dh;
+    a.mode = 0;
+    a.q_off = p.seq_offsets;
+    a.kv_off = p.seq_offsets;
+    a.q = uvqk + 2 * F;
+    a.k = uvqk + 3 * F;
+    a.v = uvqk + F;
+    a.q_stride = a.k_stride = a.v_stride = 4 * F;
+    a.total_q = a.total_kv = p.T;
+    a.out = attn;
+    a.out_stride = F;
+    a.pos_table = p.pos_table;
+    a.n_pos = p.n_pos;
+    a.time_table = p.time_table;
+    a.n_time = p.n_time;
+    a.ts = p.ts;
+    a.scale = p.scale;
+    a.max_q = a.max_kv = p.max_len;
+    e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
+    if (e != cudaSuccess) return e;
+    ln_gate_kernel<<<(unsigned)((p.T + 7) / 8), 256, 0, stream>>>(attn, uvqk, 4 * F, gate, p.T,
+                                                                  p.ln_eps);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+                                  err_word, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace hstu

@@ -27,8 +27,9 @@ def step(table, case, users_t, dtype="bf16"):
     import generative_recommender_sequence_b200 as hstu
     n_new = case.n_new
     table.alloc(users_t, dev(n_new))
-    table.append(users_t, storage(case.new_k, dtype), storage(case.new_v, dtype),
-                 dev(workloads.offsets_from_lengths(n_new)), int(max(n_new.max(), 1)))
+    if int(n_new.sum()) > 0:
+        table.append(users_t, storage(case.new_k, dtype), storage(case.new_v, dtype),
+                     dev(workloads.offsets_from_lengths(n_new)), int(n_new.max()))
     B = case.B
     max_pages = int(np.max((case.total_lengths + 31) // 32))
     lens = torch.empty(B, dtype=torch.int64, device="cuda")
