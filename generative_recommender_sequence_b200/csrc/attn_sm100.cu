@@ -57,13 +57,27 @@ constexpr uint32_t TM_O = 0, TM_S0 = 128, TM_P0 = 384;  // S1 = S0 + 128, P1 = P
 constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
 
+constexpr int NTS = 4;              // key-timestamp ring depth
+constexpr int RROW = 160;           // position-bias row per pointwise warp (32 + 127 + pad)
+
+// Key timestamps of one key tile, staged by warp 2: exact float offsets from
+// the user's first timestamp (when |offset| < 2^23 for every key), plus the
+// raw int64 values for the exact integer path.
+struct TsSlot {
+  float f[BN];
+  long long i[BN];
+  int exact;
+  int pad[3];
+};
+
 struct __align__(1024) Smem {
   uint8_t q[kTileBytes];
   uint8_t k[KST][kTileBytes];
   uint8_t v[VST][kTileBytes];
-  int64_t kts[8][BN];          // key timestamps, one copy per pointwise warp
-  float pos_tab[kMaxRab];
-  float time_tab[kMaxRab];
+  float rrow[8][RROW];         // per pointwise warp: pos bias by (row - col + 127)
+  float pos_ext[kMaxRab];      // tables with the clamp at n-1 baked in
+  float time_ext[kMaxRab];
+  TsSlot ts[NTS];
   int qt[kMaxUsers];           // query tiles per user
   uint64_t q_full, q_empty;
   uint64_t k_full[KST], k_empty[KST];
@@ -71,6 +85,7 @@ struct __align__(1024) Smem {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t o_full, o_empty;
+  uint64_t ts_full[NTS], ts_empty[NTS];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -217,6 +232,49 @@ __device__ __forceinline__ void record_timeout(const KParams& P, Smem& sm) {
   *(volatile int*)&sm.abort_flag = 1;
 }
 
+// One 32-column chunk of one score row: add the biases, mask, SiLU, pack to
+// bf16 pairs.  MASK: 0 every key visible, 1 causal (c <= qrel), 2 c < kend,
+// 3 only the candidate's own key (c == r).  TIME: 0 none, 1 float-exponent
+// bucket (exact offsets), 2 int64 bucket.  rlc[-j] is the position bias of
+// column cb + j; tx is the time table with its clamp baked in (256 entries).
+template <int MASK, int TIME>
+__device__ __forceinline__ void pw_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16], const int cb,
+                                         const float* __restrict__ rlc, const int qrel,
+                                         const int kend, const int r, const float* ktf,
+                                         const long long* kti, const float tq1,
+                                         const long long tqi, const float* tx,
+                                         const float self_rab) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    float4 kt4;
+    if (TIME == 1) kt4 = *reinterpret_cast<const float4*>(ktf + cb + j);
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = cb + j + e;
+      float x = __uint_as_float(sv[j + e]);
+      x += (MASK == 3) ? self_rab : rlc[-(j + e)];
+      if (TIME == 1) {
+        const float kt = e == 0 ? kt4.x : (e == 1 ? kt4.y : (e == 2 ? kt4.z : kt4.w));
+        const float d1 = fmaxf(tq1 - kt, 1.0f);
+        x += tx[(__float_as_uint(d1) >> 23) - 127];
+      } else if (TIME == 2) {
+        long long dt = tqi - kti[c];
+        dt = dt < 0 ? 0 : dt;
+        x += tx[63 - __clzll(dt + 1)];
+      }
+      const float h = 0.5f * x;
+      float y = fmaf(h, tanh_approx(h), h);
+      if (MASK == 1) y = (c <= qrel) ? y : 0.f;
+      if (MASK == 2) y = (c < kend) ? y : 0.f;
+      if (MASK == 3) y = (c == r) ? y : 0.f;
+      pv[e] = y;
+    }
+    pk[j >> 1] = pack_bf16x2(pv[0], pv[1]);
+    pk[(j >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+  }
+}
+
 // ------------------------------------------------------------ the kernel
 template <bool PAGED, bool CAND>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -237,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.qt[b] = (int)((nq + BM - 1) / BM);
   }
   for (int i = tid; i < kMaxRab; i += kThreads) {
-    sm.pos_tab[i] = (P.pos_table && i < P.n_pos) ? P.pos_table[i] : 0.f;
-    sm.time_tab[i] = (P.time_table && i < P.n_time) ? P.time_table[i] : 0.f;
+    sm.pos_ext[i] = P.pos_table ? P.pos_table[min(i, P.n_pos - 1)] : 0.f;
+    sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
   }
   if (tid == 0) {
     sm.abort_flag = 0;
@@ -260,6 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&sm.o_full), 1);
     mbar_init(smem_u32(&sm.o_empty), 8);
+    for (int i = 0; i < NTS; ++i) {
+      mbar_init(smem_u32(&sm.ts_full[i]), 1);
+      mbar_init(smem_u32(&sm.ts_empty[i]), 4);
+    }
     mbar_init(smem_u32(&sm.mma_done), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -442,6 +504,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(smem_u32(&sm.mma_done), 0);
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // =============================================== key-timestamp producer
+    // Stages the key timestamps of every tile (in the MMA's tile order) for the
+    // time-gap bias, so the pointwise warps never wait on global loads.
+    if (P.time_table != nullptr && !PAGED && !CAND) {
+      Sched sc;
+      sc.init(sm.qt, P.B, HS, lane);
+      uint32_t g = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; ok; t += gridDim.x) {
+        int b, m, rem;
+        if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
+        const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+        if (it.t0 >= it.t1) continue;
+        const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
+        for (int tile = it.t0; tile < it.t1; ++tile, ++g) {
+          const uint32_t slot = g % NTS;
+          ok = mbar_wait_warp(smem_u32(&sm.ts_empty[slot]), ((g / NTS) & 1) ^ 1);
+          if (!ok) break;
+          TsSlot& ts = sm.ts[slot];
+          bool exact = true;
+#pragma unroll
+          for (int i = 0; i < BN / 32; ++i) {
+            const int c = lane + 32 * i;
+            const int64_t kp = (int64_t)tile * BN + c;
+            long long v = base;
+            if (kp < it.n_k) v = P.ts[it.kv_row0 + kp];
+            const long long rel = v - base;
+            exact = exact && rel > -(1LL << 23) && rel < (1LL << 23);
+            ts.i[c] = v;
+            ts.f[c] = (float)rel;
+          }
+          exact = __all_sync(0xffffffffu, exact);
+          if (lane == 0) ts.exact = exact ? 1 : 0;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.ts_full[slot]));
+        }
+      }
+      if (!ok && lane == 0) record_timeout(P, sm);
+    }
   } else if (warp >= 4) {
     // =============================================== pointwise + epilogue
     const int wg = (warp - 4) >> 2;                 // 0 or 1
@@ -449,11 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = sub * 32 + lane;                  // tile row owned by this thread
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
+    const bool use_pos = P.pos_table != nullptr;
+    float* rrow = sm.rrow[warp - 4];
     Sched sc;
     sc.init(sm.qt, P.B, HS, lane);
     uint32_t qi = 0, g = 0;
     bool ok = true;
-    int64_t* kts = sm.kts[warp - 4];
     for (long long t = blockIdx.x; ok; t += gridDim.x) {
       int b, m, rem;
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
@@ -461,12 +564,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
-      int64_t ts_q = 0;
-      if (use_time) {
-        const int64_t qpc = min64(max64(qp, 0), max64(it.n_k - 1, 0));
-        ts_q = it.n_k > 0 ? P.ts[it.kv_row0 + qpc] : 0;
+      long long tq_i = 0;
+      float tq1 = 1.f;
+      bool tq_exact = true;
+      if (use_time && it.n_k > 0) {
+        const long long base = P.ts[it.kv_row0];
+        if (r < it.nvalid) {
+          const int64_t qpc = min64(max64(qp, 0), it.n_k - 1);
+          tq_i = P.ts[it.kv_row0 + qpc];
+        } else {
+          tq_i = base;
+        }
+        const long long rel = tq_i - base;
+        tq_exact = rel > -(1LL << 23) && rel < (1LL << 23);
+        tq1 = (float)rel + 1.f;
       }
-      const int n_pos_m1 = P.n_pos - 1, n_time_m1 = P.n_time - 1;
+      tq_exact = __all_sync(0xffffffffu, tq_exact);
       for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
         if ((int)(g & 1) != wg) continue;
         const uint32_t sb = g & 1;
@@ -474,77 +587,103 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
         // int32 tile-relative coordinates: query position minus k0, valid keys
         const int qrel = (int)max64(min64(qp - k0, 1 << 30), -(1 << 30));
+        const int qrel0 = __shfl_sync(0xffffffffu, qrel, 0);  // smallest in the warp
         const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
-        if (use_time) {
+        // position-bias row of this warp: rrow[j] = pos bias at delta qrel0 + j - 127
+        if (use_pos && !cand_tile) {
           __syncwarp();
-          for (int i = lane; i < BN; i += 32) {
-            const int64_t kp = k0 + i;
-            kts[i] = kp < it.n_k ? P.ts[it.kv_row0 + kp] : 0;
+#pragma unroll
+          for (int i = 0; i < RROW / 32; ++i) {
+            const int j = lane + 32 * i;
+            const int delta = max(qrel0 + j - 127, 0);
+            rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
           }
           __syncwarp();
+        }
+        const float* rl = use_pos ? (CAND ? rrow : rrow + lane) : sm.pos_ext;  // zeros without a table
+        const uint32_t tslot = g % NTS;
+        bool time_fast = false;
+        if (use_time) {
+          ok = mbar_wait_warp(smem_u32(&sm.ts_full[tslot]), (g / NTS) & 1);
+          if (!ok) break;
+          time_fast = tq_exact && sm.ts[tslot].exact;
         }
         ok = mbar_wait_warp(smem_u32(&sm.s_full[sb]), (g >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_addr + TM_S0 + sb * 128;
         const uint32_t p_addr = tmem + lane_addr + TM_P0 + sb * 64;
+        const float self_rab = sm.pos_ext[0];
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
-          uint32_t sa[32], sb2[32];
-          tmem_ld32(s_addr + half * 64, sa);
-          tmem_ld32(s_addr + half * 64 + 32, sb2);
+          uint32_t sv[2][32];
+          tmem_ld32(s_addr + half * 64, sv[0]);
+          tmem_ld32(s_addr + half * 64 + 32, sv[1]);
           tmem_wait_ld();
-          reg_fence(sa);
-          reg_fence(sb2);
+          reg_fence(sv[0]);
+          reg_fence(sv[1]);
           if (half == 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
           }
-          uint32_t packed[32];
+          uint32_t pk[2][16];
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            float pv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = half * 64 + j + e;
-              const float s = __uint_as_float(j + e < 32 ? sa[j + e] : sb2[j + e - 32]);
-              bool valid;
-              int delta;
-              if (CAND) {
-                valid = cand_tile ? (c == r) : (c < kend);
-                delta = cand_tile ? 0 : qrel - c;
+          for (int q = 0; q < 2; ++q) {
+            const int cb = half * 64 + q * 32;
+            // warp-uniform mask class of this 32-column chunk
+            int cls;  // 0 visible, 1 per-element, 2 none visible
+            int mk;   // per-element mask kind
+            if (CAND) {
+              if (cand_tile) {
+                cls = (cb == 32 * sub) ? 1 : 2;
+                mk = 3;
               } else {
-                valid = c <= qrel;
-                delta = qrel - c;
+                cls = (cb + 31 < kend) ? 0 : (cb >= kend ? 2 : 1);
+                mk = 2;
               }
-              const int bk = 31 - __clz(max(delta, 0) + 1);
-              float x = s + sm.pos_tab[min(bk, n_pos_m1)];
-              if (use_time) {
-                long long dt = ts_q - kts[c];
-                dt = dt < 0 ? 0 : dt;
-                const int bt = 63 - __clzll(dt + 1);
-                x += sm.time_tab[min(bt, n_time_m1)];
-              }
-              const float hx = 0.5f * x;
-              const float y = fmaf(hx, tanh_approx(hx), hx);
-              pv[e] = valid ? y : 0.f;
+            } else {
+              cls = (cb + 31 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
+              mk = 1;
             }
-            packed[j >> 1] = pack_bf16x2(pv[0], pv[1]);
+            const float* rlc = rl + 127 - cb;
+            if (cls == 2) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pk[q][j] = 0u;
+            } else if (use_time) {
+              const TsSlot& ts = sm.ts[tslot];
+              if (time_fast) {
+                if (cls == 0)
+                  pw_chunk<0, 1>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                else
+                  pw_chunk<1, 1>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+              } else {
+                if (cls == 0)
+                  pw_chunk<0, 2>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                else
+                  pw_chunk<1, 2>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+              }
+            } else if (cls == 0) {
+              pw_chunk<0, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+            } else if (mk == 1) {
+              pw_chunk<1, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+            } else if (mk == 2) {
+              pw_chunk<2, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+            } else {
+              pw_chunk<3, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+            }
+          }
+          if (half == 1 && use_time) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
           }
           if (half == 0) {
             ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
             if (!ok) break;
             tc_fence_after();
           }
-          uint32_t lo[16], hi[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            lo[j] = packed[j];
-            hi[j] = packed[16 + j];
-          }
-          tmem_st16(p_addr + half * 32, lo);
-          tmem_st16(p_addr + half * 32 + 16, hi);
+          tmem_st16(p_addr + half * 32, pk[0]);
+          tmem_st16(p_addr + half * 32 + 16, pk[1]);
         }
         if (!ok) break;
         tmem_wait_st();
