@@ -44,7 +44,8 @@ namespace {
 constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
 constexpr int HD = 128;            // head dim
-constexpr int KST = 3;             // K ring depth
+constexpr int KST = 2;             // K ring depth
+constexpr int QST = 2;             // Q double buffer (next item's Q loads early)
 constexpr int VST = 2;             // V ring depth
 constexpr int kThreads = 384;
 constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
@@ -71,7 +72,7 @@ struct TsSlot {
 };
 
 struct __align__(1024) Smem {
-  uint8_t q[kTileBytes];
+  uint8_t q[QST][kTileBytes];
   uint8_t k[KST][kTileBytes];
   uint8_t v[VST][kTileBytes];
   float rrow[8][RROW];         // per pointwise warp: pos bias by (row - col + 127)
@@ -79,7 +80,7 @@ struct __align__(1024) Smem {
   float time_ext[kMaxRab];
   TsSlot ts[NTS];
   int qt[kMaxUsers];           // query tiles per user
-  uint64_t q_full, q_empty;
+  uint64_t q_full[QST], q_empty[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[2], s_empty[2];
@@ -300,8 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     sm.abort_flag = 0;
-    mbar_init(smem_u32(&sm.q_full), 1);
-    mbar_init(smem_u32(&sm.q_empty), 1);
+    for (int i = 0; i < QST; ++i) {
+      mbar_init(smem_u32(&sm.q_full[i]), 1);
+      mbar_init(smem_u32(&sm.q_empty[i]), 1);
+    }
     for (int i = 0; i < KST; ++i) {
       mbar_init(smem_u32(&sm.k_full[i]), 1);
       mbar_init(smem_u32(&sm.k_empty[i]), 1);
@@ -354,12 +357,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
-        ok = mbar_wait(smem_u32(&sm.q_empty), (qi & 1) ^ 1);
+        const uint32_t qs = qi % QST;
+        ok = mbar_wait(smem_u32(&sm.q_empty[qs]), ((qi / QST) & 1) ^ 1);
         if (ok) {
-          const uint32_t bar = smem_u32(&sm.q_full);
+          const uint32_t bar = smem_u32(&sm.q_full[qs]);
           mbar_arrive_expect_tx(bar, kTileBytes);
-          tma_load_3d(smem_u32(sm.q), &tm_q, bar, 0, it.h, (int)it.q_row0);
-          tma_load_3d(smem_u32(sm.q) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
+          tma_load_3d(smem_u32(sm.q[qs]), &tm_q, bar, 0, it.h, (int)it.q_row0);
+          tma_load_3d(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -428,7 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t c = vc - 1 - i;
         mbar_wait(smem_u32(&sm.v_full[c % VST]), (c / VST) & 1);
       }
-      if (qi > 0) mbar_wait(smem_u32(&sm.q_full), (qi - 1) & 1);
+      for (uint32_t i = 0; i < QST && i < qi; ++i) {
+        const uint32_t c = qi - 1 - i;
+        mbar_wait(smem_u32(&sm.q_full[c % QST]), (c / QST) & 1);
+      }
     }
   } else if (warp == 1) {
     // =============================================== MMA issuer
@@ -436,7 +443,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.init(sm.qt, P.B, HS, lane);
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
-    const uint32_t q_base = smem_u32(sm.q);
+    auto issue_qk = [&](uint32_t gq, uint32_t q_base) -> bool {
+      const uint32_t sb = gq & 1;
+      if (!mbar_wait(smem_u32(&sm.s_empty[sb]), ((gq >> 1) & 1) ^ 1)) return false;
+      const uint32_t slot = kc % KST;
+      if (!mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1)) return false;
+      tc_fence_after();
+      const uint32_t k_base = smem_u32(sm.k[slot]);
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+        const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+        umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(smem_u32(&sm.k_empty[slot]));
+      umma_commit(smem_u32(&sm.s_full[sb]));
+      ++kc;
+      return true;
+    };
     auto issue_pv = [&](uint32_t gp, bool first) -> bool {
       const uint32_t pb = gp & 1;
       if (!mbar_wait(smem_u32(&sm.p_full[pb]), (gp >> 1) & 1)) return false;
@@ -458,37 +483,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++vc;
       return true;
     };
+    // Per item: S = Q K^T runs two key tiles ahead of O += P V, so the next
+    // S of a warpgroup is ready when it finishes its current tile (the S
+    // buffer frees as soon as the warpgroup has loaded it).
     for (long long t = blockIdx.x; ok; t += gridDim.x) {
       int b, m, rem;
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
-        ok = mbar_wait(smem_u32(&sm.q_full), qi & 1);
+        const uint32_t qs = qi % QST;
+        const uint32_t q_base = smem_u32(sm.q[qs]);
+        ok = mbar_wait(smem_u32(&sm.q_full[qs]), (qi / QST) & 1);
         const int nt = it.t1 - it.t0;
+        const uint32_t g0 = g;
+        for (int i = 0; i < 2 && i < nt && ok; ++i) ok = issue_qk(g0 + i, q_base);
+        if (ok && nt <= 2) umma_commit(smem_u32(&sm.q_empty[qs]));
         for (int i = 0; i < nt && ok; ++i) {
-          const uint32_t sb = g & 1;
-          ok = mbar_wait(smem_u32(&sm.s_empty[sb]), ((g >> 1) & 1) ^ 1);
-          const uint32_t slot = kc % KST;
-          if (ok) ok = mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(sm.k[slot]);
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-            umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+          if (i + 2 < nt) {
+            ok = issue_qk(g0 + i + 2, q_base);
+            if (ok && i + 2 == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
           }
-          umma_commit(smem_u32(&sm.k_empty[slot]));
-          umma_commit(smem_u32(&sm.s_full[sb]));
-          ++kc;
-          if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty));
-          if (i > 0) ok = issue_pv(g - 1, i == 1);
-          ++g;
+          if (ok) ok = issue_pv(g0 + i, i == 0);
         }
-        if (ok) ok = issue_pv(g - 1, nt == 1);
+        g = g0 + nt;
         if (ok) umma_commit(smem_u32(&sm.o_full));
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
