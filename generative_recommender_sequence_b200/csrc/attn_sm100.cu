@@ -13,16 +13,18 @@
 // recommandeurs génératifs avec NVIDIA Dynamo-Triton et HSTU", section
 // "Comment cela fonctionne").
 //
-// Structure (one persistent CTA per SM, 384 threads):
-//   warp 0      TMA producer: Q tile (128 x 128), K ring (3 x 128 x 128),
+// Structure (one persistent CTA per SM, 640 threads):
+//   warp 0      TMA producer: Q tile (128 x 128), K ring (2 x 128 x 128), Q double buffer,
 //               V ring (2 x 128 x 128), all 128-byte swizzled.  Paged keys are
 //               four 32-token page boxes per 128-key tile.
 //   warp 1      tcgen05 issuer: S = Q K^T into TMEM (two S buffers), then
 //               O += P V with P read from TMEM (two bf16 P buffers).
-//   warps 4-11  two "pointwise" warpgroups, alternating key tiles: read S
-//               from TMEM, add the bias, apply the mask, SiLU (via tanh), pack P
-//               to bf16 in TMEM; then the epilogue (O * scale -> bf16 or fp32
-//               split partial).
+//   warp 2      stages key timestamps for the time-gap bias (mbarrier ring)
+//   warps 4-19  four "pointwise" warpgroups: two pairs alternate key tiles, the
+//               two warpgroups of a pair split the tile's 128 score columns;
+//               read S from TMEM, add the biases, mask, SiLU (via tanh), pack
+//               P to bf16 in TMEM; then the epilogue (O * scale -> bf16 or fp32
+//               split partial), 32 output columns per warpgroup.
 // There is no softmax, so there is no running max and no rescaling of O, and
 // key splits of one query tile add exactly (the candidate path splits keys).
 // Work items (user, head, query tile, split) run longest-first: query tiles
@@ -47,7 +49,7 @@ constexpr int HD = 128;            // head dim
 constexpr int KST = 2;             // K ring depth
 constexpr int QST = 2;             // Q double buffer (next item's Q loads early)
 constexpr int VST = 2;             // V ring depth
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;      // 20 warps: TMA, MMA, timestamps, spare, 16 pointwise
 constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
 constexpr int kMaxUsers = 2048;
@@ -75,7 +77,7 @@ struct __align__(1024) Smem {
   uint8_t q[QST][kTileBytes];
   uint8_t k[KST][kTileBytes];
   uint8_t v[VST][kTileBytes];
-  float rrow[8][RROW];         // per pointwise warp: pos bias by (row - col + 127)
+  float rrow[16][RROW];        // per pointwise warp: pos bias by (row - col + 127)
   float pos_ext[kMaxRab];      // tables with the clamp at n-1 baked in
   float time_ext[kMaxRab];
   TsSlot ts[NTS];
@@ -315,15 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_empty[i]), 4);
-      mbar_init(smem_u32(&sm.p_full[i]), 4);
+      mbar_init(smem_u32(&sm.s_empty[i]), 8);
+      mbar_init(smem_u32(&sm.p_full[i]), 8);
       mbar_init(smem_u32(&sm.p_empty[i]), 1);
     }
     mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.o_empty), 8);
+    mbar_init(smem_u32(&sm.o_empty), 16);
     for (int i = 0; i < NTS; ++i) {
       mbar_init(smem_u32(&sm.ts_full[i]), 1);
-      mbar_init(smem_u32(&sm.ts_empty[i]), 4);
+      mbar_init(smem_u32(&sm.ts_empty[i]), 8);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
     fence_mbar_init();
@@ -564,13 +566,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // =============================================== pointwise + epilogue
-    const int wg = (warp - 4) >> 2;                 // 0 or 1
+    // 16 warps: key tiles alternate between two pairs of warpgroups; within a
+    // pair, warpgroup `chalf` takes score columns [64 chalf, 64 chalf + 64).
+    const int pwi = warp - 4;                       // 0..15
+    const int wg = pwi >> 3;                        // tile parity handled
+    const int chalf = (pwi >> 2) & 1;               // column half of the tile
+    const int ocol = (pwi >> 2) * 32;               // epilogue: O columns [ocol, ocol + 32)
     const int sub = warp & 3;                       // TMEM lane quarter
     const int r = sub * 32 + lane;                  // tile row owned by this thread
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
     const bool use_pos = P.pos_table != nullptr;
-    float* rrow = sm.rrow[warp - 4];
+    float* rrow = sm.rrow[pwi];
     Sched sc;
     sc.init(sm.qt, P.B, HS, lane);
     uint32_t qi = 0, g = 0;
@@ -632,23 +639,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_addr = tmem + lane_addr + TM_S0 + sb * 128;
         const uint32_t p_addr = tmem + lane_addr + TM_P0 + sb * 64;
         const float self_rab = sm.pos_ext[0];
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sv[2][32];
-          tmem_ld32(s_addr + half * 64, sv[0]);
-          tmem_ld32(s_addr + half * 64 + 32, sv[1]);
-          tmem_wait_ld();
-          reg_fence(sv[0]);
-          reg_fence(sv[1]);
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
-          }
+        {
+          const int half = chalf;
           uint32_t pk[2][16];
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             const int cb = half * 64 + q * 32;
+            uint32_t sv[32];
+            tmem_ld32(s_addr + cb, sv);
+            tmem_wait_ld();
+            reg_fence(sv);
+            if (q == 1) {  // this warp's part of S is in registers: the buffer may be rewritten
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+            }
             // warp-uniform mask class of this 32-column chunk
             int cls;  // 0 visible, 1 per-element, 2 none visible
             int mk;   // per-element mask kind
@@ -672,34 +677,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               const TsSlot& ts = sm.ts[tslot];
               if (time_fast) {
                 if (cls == 0)
-                  pw_chunk<0, 1>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                  pw_chunk<0, 1>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
                 else
-                  pw_chunk<1, 1>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                  pw_chunk<1, 1>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
               } else {
                 if (cls == 0)
-                  pw_chunk<0, 2>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                  pw_chunk<0, 2>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
                 else
-                  pw_chunk<1, 2>(sv[q], pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
+                  pw_chunk<1, 2>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
               }
             } else if (cls == 0) {
-              pw_chunk<0, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+              pw_chunk<0, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
             } else if (mk == 1) {
-              pw_chunk<1, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+              pw_chunk<1, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
             } else if (mk == 2) {
-              pw_chunk<2, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+              pw_chunk<2, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
             } else {
-              pw_chunk<3, 0>(sv[q], pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+              pw_chunk<3, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
             }
           }
-          if (half == 1 && use_time) {
+          if (use_time) {
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
           }
-          if (half == 0) {
-            ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
-            if (!ok) break;
-            tc_fence_after();
-          }
+          ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
+          if (!ok) break;
+          tc_fence_after();
           tmem_st16(p_addr + half * 32, pk[0]);
           tmem_st16(p_addr + half * 32 + 16, pk[1]);
         }
@@ -710,17 +713,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       }
       if (!ok) break;
-      // ---- epilogue: this warpgroup stores columns [64 wg, 64 wg + 64)
+      // ---- epilogue: this warpgroup stores O columns [ocol, ocol + 32)
       ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
       if (!ok) break;
       tc_fence_after();
-      uint32_t oa[32], ob[32];
-      const uint32_t o_addr = tmem + lane_addr + TM_O + wg * 64;
-      tmem_ld32(o_addr, oa);
-      tmem_ld32(o_addr + 32, ob);
+      uint32_t oa[32];
+      tmem_ld32(tmem + lane_addr + TM_O + ocol, oa);
       tmem_wait_ld();
       reg_fence(oa);
-      reg_fence(ob);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
@@ -729,32 +729,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t row = it.q_row0 + r;
         if (P.partial) {
           float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
-                       it.h * HD + wg * 64;
+                       it.h * HD + ocol;
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
+          for (int j = 0; j < 32; j += 4)
             reinterpret_cast<float4*>(dst)[j / 4] =
                 make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
                             __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
-            reinterpret_cast<float4*>(dst + 32)[j / 4] =
-                make_float4(__uint_as_float(ob[j]), __uint_as_float(ob[j + 1]),
-                            __uint_as_float(ob[j + 2]), __uint_as_float(ob[j + 3]));
-          }
         } else {
-          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + wg * 64;
+          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + ocol;
           const float sc2 = P.scale;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
-            uint4 u, w;
+            uint4 u;
             u.x = pack_bf16x2(__uint_as_float(oa[j]) * sc2, __uint_as_float(oa[j + 1]) * sc2);
             u.y = pack_bf16x2(__uint_as_float(oa[j + 2]) * sc2, __uint_as_float(oa[j + 3]) * sc2);
             u.z = pack_bf16x2(__uint_as_float(oa[j + 4]) * sc2, __uint_as_float(oa[j + 5]) * sc2);
             u.w = pack_bf16x2(__uint_as_float(oa[j + 6]) * sc2, __uint_as_float(oa[j + 7]) * sc2);
-            w.x = pack_bf16x2(__uint_as_float(ob[j]) * sc2, __uint_as_float(ob[j + 1]) * sc2);
-            w.y = pack_bf16x2(__uint_as_float(ob[j + 2]) * sc2, __uint_as_float(ob[j + 3]) * sc2);
-            w.z = pack_bf16x2(__uint_as_float(ob[j + 4]) * sc2, __uint_as_float(ob[j + 5]) * sc2);
-            w.w = pack_bf16x2(__uint_as_float(ob[j + 6]) * sc2, __uint_as_float(ob[j + 7]) * sc2);
             reinterpret_cast<uint4*>(dst)[j / 8] = u;
-            reinterpret_cast<uint4*>(dst + 32)[j / 8] = w;
           }
         }
       }
