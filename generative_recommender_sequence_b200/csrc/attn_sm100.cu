@@ -17,8 +17,8 @@
 //   warp 0      TMA producer: Q tile (128 x 128), K ring (2 x 128 x 128), Q double buffer,
 //               V ring (2 x 128 x 128), all 128-byte swizzled.  Paged keys are
 //               four 32-token page boxes per 128-key tile.
-//   warp 1      tcgen05 issuer: S = Q K^T into TMEM (two S buffers), then
-//               O += P V with P read from TMEM (two bf16 P buffers).
+//   warp 1      tcgen05 issuer of S = Q K^T into TMEM (two S buffers)
+//   warp 3      tcgen05 issuer of O += P V, P read from TMEM (two bf16 P buffers)
 //   warp 2      stages key timestamps for the time-gap bias (mbarrier ring)
 //   warps 4-19  four "pointwise" warpgroups: two pairs alternate key tiles, the
 //               two warpgroups of a pair split the tile's 128 score columns;
@@ -89,7 +89,7 @@ struct __align__(1024) Smem {
   uint64_t p_full[2], p_empty[2];
   uint64_t o_full, o_empty;
   uint64_t ts_full[NTS], ts_empty[NTS];
-  uint64_t mma_done;
+  uint64_t mma_done, mma_done2;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -174,6 +174,14 @@ struct Sched {
     return b >= 0;
   }
 };
+
+// Items are sorted longest first; round k hands them to the CTAs in forward
+// order for even k and in reverse order for odd k (a snake), so the CTA that
+// got the longest item of one round gets the shortest of the next.
+__device__ __forceinline__ long long snake_item(long long rnd) {
+  const long long G = gridDim.x;
+  return rnd * G + ((rnd & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
+}
 
 struct Item {
   int b, h, m, s;
@@ -328,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.ts_empty[i]), 8);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
+    mbar_init(smem_u32(&sm.mma_done2), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -353,7 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.init(sm.qt, P.B, HS, lane);
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
-    for (long long t = blockIdx.x;; t += gridDim.x) {
+    for (long long rnd = 0;; ++rnd) {
+      const long long t = snake_item(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
@@ -439,89 +449,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(smem_u32(&sm.q_full[c % QST]), (c / QST) & 1);
       }
     }
-  } else if (warp == 1) {
-    // =============================================== MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // =============================================== MMA issuers
+    // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
+    // tensor pipe fed: while one waits on its barriers the other's MMAs run.
     Sched sc;
     sc.init(sm.qt, P.B, HS, lane);
+    const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
-    auto issue_qk = [&](uint32_t gq, uint32_t q_base) -> bool {
-      const uint32_t sb = gq & 1;
-      if (!mbar_wait(smem_u32(&sm.s_empty[sb]), ((gq >> 1) & 1) ^ 1)) return false;
-      const uint32_t slot = kc % KST;
-      if (!mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1)) return false;
-      tc_fence_after();
-      const uint32_t k_base = smem_u32(sm.k[slot]);
-#pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-        const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-        umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(smem_u32(&sm.k_empty[slot]));
-      umma_commit(smem_u32(&sm.s_full[sb]));
-      ++kc;
-      return true;
-    };
-    auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-      const uint32_t pb = gp & 1;
-      if (!mbar_wait(smem_u32(&sm.p_full[pb]), (gp >> 1) & 1)) return false;
-      const uint32_t slot = vc % VST;
-      if (!mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1)) return false;
-      if (first && !mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1)) return false;
-      tc_fence_after();
-      const uint32_t v_base = smem_u32(sm.v[slot]);
-#pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key groups
-        // 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
-        const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
-        umma_ts(tmem + TM_O, tmem + TM_P0 + pb * 64 + kk * 8, bdesc, kIdescPV,
-                (first && kk == 0) ? 0u : 1u);
-      }
-      umma_commit(smem_u32(&sm.v_empty[slot]));
-      umma_commit(smem_u32(&sm.p_empty[pb]));
-      ++vc;
-      return true;
-    };
-    // Per item: S = Q K^T runs two key tiles ahead of O += P V, so the next
-    // S of a warpgroup is ready when it finishes its current tile (the S
-    // buffer frees as soon as the warpgroup has loaded it).
-    for (long long t = blockIdx.x; ok; t += gridDim.x) {
+    for (long long rnd = 0; ok; ++rnd) {
+      const long long t = snake_item(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
       if (it.t0 >= it.t1) continue;
+      const int nt = it.t1 - it.t0;
       if (lane == 0) {
-        const uint32_t qs = qi % QST;
-        const uint32_t q_base = smem_u32(sm.q[qs]);
-        ok = mbar_wait(smem_u32(&sm.q_full[qs]), (qi / QST) & 1);
-        const int nt = it.t1 - it.t0;
-        const uint32_t g0 = g;
-        for (int i = 0; i < 2 && i < nt && ok; ++i) ok = issue_qk(g0 + i, q_base);
-        if (ok && nt <= 2) umma_commit(smem_u32(&sm.q_empty[qs]));
-        for (int i = 0; i < nt && ok; ++i) {
-          if (i + 2 < nt) {
-            ok = issue_qk(g0 + i + 2, q_base);
-            if (ok && i + 2 == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
+        if (qk_role) {
+          const uint32_t qs = qi % QST;
+          const uint32_t q_base = smem_u32(sm.q[qs]);
+          ok = mbar_wait(smem_u32(&sm.q_full[qs]), (qi / QST) & 1);
+          for (int i = 0; i < nt && ok; ++i, ++g, ++kc) {
+            const uint32_t sb = g & 1;
+            const uint32_t slot = kc % KST;
+            ok = mbar_wait(smem_u32(&sm.s_empty[sb]), ((g >> 1) & 1) ^ 1) &&
+                 mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sm.k[slot]);
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+              const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+              umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&sm.k_empty[slot]));
+            umma_commit(smem_u32(&sm.s_full[sb]));
+            if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
           }
-          if (ok) ok = issue_pv(g0 + i, i == 0);
+        } else {
+          for (int i = 0; i < nt && ok; ++i, ++g, ++vc) {
+            const uint32_t pb = g & 1;
+            const uint32_t slot = vc % VST;
+            ok = mbar_wait(smem_u32(&sm.p_full[pb]), (g >> 1) & 1) &&
+                 mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1) &&
+                 (i != 0 || mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(sm.v[slot]);
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key
+              // groups 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
+              const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
+              umma_ts(tmem + TM_O, tmem + TM_P0 + pb * 64 + kk * 8, bdesc, kIdescPV,
+                      (i == 0 && kk == 0) ? 0u : 1u);
+            }
+            umma_commit(smem_u32(&sm.v_empty[slot]));
+            umma_commit(smem_u32(&sm.p_empty[pb]));
+          }
+          if (ok) umma_commit(smem_u32(&sm.o_full));
         }
-        g = g0 + nt;
-        if (ok) umma_commit(smem_u32(&sm.o_full));
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       g = __shfl_sync(0xffffffffu, g, 0);
-      kc = __shfl_sync(0xffffffffu, kc, 0);
-      vc = __shfl_sync(0xffffffffu, vc, 0);
       ++qi;
     }
     if (lane == 0) {
       if (!ok) record_timeout(P, sm);
       // all MMAs issued by this thread must finish before TMEM is released
-      umma_commit(smem_u32(&sm.mma_done));
-      mbar_wait(smem_u32(&sm.mma_done), 0);
+      const uint32_t done = smem_u32(qk_role ? &sm.mma_done : &sm.mma_done2);
+      umma_commit(done);
+      mbar_wait(done, 0);
     }
     __syncwarp();
   } else if (warp == 2) {
@@ -533,7 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc.init(sm.qt, P.B, HS, lane);
       uint32_t g = 0;
       bool ok = true;
-      for (long long t = blockIdx.x; ok; t += gridDim.x) {
+      for (long long rnd = 0; ok; ++rnd) {
+      const long long t = snake_item(rnd);
         int b, m, rem;
         if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
         const Item it = make_item<PAGED, CAND>(P, b, m, rem);
@@ -582,7 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.init(sm.qt, P.B, HS, lane);
     uint32_t qi = 0, g = 0;
     bool ok = true;
-    for (long long t = blockIdx.x; ok; t += gridDim.x) {
+    for (long long rnd = 0; ok; ++rnd) {
+      const long long t = snake_item(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND>(P, b, m, rem);
