@@ -55,6 +55,9 @@ _SIGNATURES = {
     "hstu_attn_cached_fwd": ([_P, _P, _I32, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _F, _P, _P,
                               _SZ, _P], _I32),
     "hstu_attn_cached_workspace_size": ([_P, _I32, _I64, _I32, _I32, _I32], _SZ),
+    "hstu_attn_cached_noalloc_max_scratch": ([], _SZ),
+    "hstu_attn_cached_fwd_noalloc": ([_P, _P, _I32, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _F, _P,
+                                      _P], _I32),
     "hstu_block_fwd": ([_P, _P, _I32, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _F, _F, _P,
                         _SZ, _P], _I32),
     "hstu_block_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),

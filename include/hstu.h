@@ -202,6 +202,28 @@ HSTU_API size_t hstu_attn_cached_workspace_size(hstu_kv_table* t, int32_t B, int
                                        int32_t max_q, int32_t max_cached, int32_t mask_mode);
 
 /*
+ * Allocation-free variant of hstu_attn_cached_fwd (no counterpart on the pages:
+ * it exists for callers that cannot allocate device memory on their request
+ * path, such as a server whose allocator is frozen after warm-up or code that
+ * runs inside someone else's memory pool).  Same arguments and results as
+ * hstu_attn_cached_fwd without workspace/ws_bytes: the split partial sums go
+ * to a fixed array of hstu_attn_cached_noalloc_max_scratch() bytes (32 MiB)
+ * that the library reserves on every GPU where it is loaded, kept until the
+ * process exits.  Calls needing more than that return HSTU_ERR_UNSUPPORTED.
+ * The first call on a device looks the array's address up (with that device
+ * current) and should come before any stream capture.  All calls share the
+ * array: calls that overlap on the GPU race, so do not run two at once.
+ * Allocates no memory.
+ */
+HSTU_API size_t hstu_attn_cached_noalloc_max_scratch(void);
+HSTU_API hstu_status hstu_attn_cached_fwd_noalloc(hstu_kv_table* t, const int64_t* users, int32_t B,
+                                                  const void* q, const void* k_cand,
+                                                  const void* v_cand, const int64_t* q_offsets,
+                                                  int64_t total_q, int32_t max_q, int32_t max_cached,
+                                                  int32_t mask_mode, const hstu_rab* rab, float scale,
+                                                  void* out, cudaStream_t stream);
+
+/*
  * HSTU block stack ("HSTU" section: projection, SiLU, SiLU attention with rab,
  * elementwise gate before the output projection), bf16 with fp32 accumulation:
  *   for each layer l:
