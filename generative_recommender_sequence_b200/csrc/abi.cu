@@ -195,7 +195,6 @@ hstu_status hstu_attn_fwd(const void* q, const void* k, const void* v, const int
   if (dt == HSTU_BF16 && d_qk == 128) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
       return HSTU_ERR_INVALID_ARG;
-    if (B > 2048) return HSTU_ERR_UNSUPPORTED;
   }
   if (B == 0 || max_len == 0 || total_tokens == 0) return HSTU_OK;
   AttnProblem p;
@@ -392,7 +391,6 @@ hstu_status hstu_attn_cached_fwd(hstu_kv_table* t, const int64_t* users, int32_t
   if (!p.f32 && p.d == 128) {
     if (!aligned16(q) || !aligned16(out) || (k_cand && (!aligned16(k_cand) || !aligned16(v_cand))))
       return HSTU_ERR_INVALID_ARG;
-    if (B > 2048) return HSTU_ERR_UNSUPPORTED;
     const size_t need = attn_sm100_workspace_bytes(p, device_sm_count());
     if (need > 0 && (workspace == nullptr || ws_bytes < need)) return HSTU_ERR_INVALID_ARG;
   }
@@ -417,7 +415,6 @@ hstu_status hstu_block_fwd(void* x, const int64_t* seq_offsets, int32_t B, int32
     return HSTU_ERR_INVALID_ARG;
   if (T >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
   if (dh != 128 || H * dh != d_model || d_model % 128 != 0) return HSTU_ERR_UNSUPPORTED;
-  if (B > 2048) return HSTU_ERR_UNSUPPORTED;
   if (!rab_ok(rab, true)) return HSTU_ERR_INVALID_ARG;
   if (T == 0 || n_layers == 0 || B == 0) return HSTU_OK;
   if (!x || !seq_offsets || !w_uvqk || !w_o || !aligned16(x)) return HSTU_ERR_INVALID_ARG;

@@ -52,7 +52,7 @@ constexpr int VST = 2;             // V ring depth
 constexpr int kThreads = 640;      // 20 warps: TMA, MMA, timestamps, spare, 16 pointwise
 constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
-constexpr int kMaxUsers = 2048;
+constexpr int kMaxUsers = 1024;   // per launch; larger batches are split on the host
 constexpr int kMaxRab = 256;
 
 constexpr uint32_t TM_O = 0, TM_S0 = 128, TM_P0 = 384;  // S1 = S0 + 128, P1 = P0 + 64
@@ -61,7 +61,8 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
 
 constexpr int NTS = 4;              // key-timestamp ring depth
-constexpr int RROW = 160;           // position-bias row per pointwise warp (32 + 127 + pad)
+constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
+constexpr int RROW = 96;            // position-bias row per pointwise warp (its 64 columns + 31)
 
 // Key timestamps of one key tile, staged by warp 2: exact float offsets from
 // the user's first timestamp (when |offset| < 2^23 for every key), plus the
@@ -77,11 +78,15 @@ struct __align__(1024) Smem {
   uint8_t q[QST][kTileBytes];
   uint8_t k[KST][kTileBytes];
   uint8_t v[VST][kTileBytes];
-  float rrow[16][RROW];        // per pointwise warp: pos bias by (row - col + 127)
+  float rrow[16][RROW];        // per pointwise warp: pos bias by (row - col), its column half
   float pos_ext[kMaxRab];      // tables with the clamp at n-1 baked in
   float time_ext[kMaxRab];
   TsSlot ts[NTS];
-  int qt[kMaxUsers];           // query tiles per user
+  int m_q[kMaxUsers + 1];      // per user: first query row
+  int m_kv[kMaxUsers];         // per user: first key row (contiguous) or user id (paged)
+  int m_nk[kMaxUsers];         // per user: number of keys (sequence / cached length)
+  TsSlot qts[2];               // query timestamps of the current / next item
+  int pages[kPagesStaged];     // producer: page ids of the current item's key tiles
   uint64_t q_full[QST], q_empty[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
@@ -89,6 +94,7 @@ struct __align__(1024) Smem {
   uint64_t p_full[2], p_empty[2];
   uint64_t o_full, o_empty;
   uint64_t ts_full[NTS], ts_empty[NTS];
+  uint64_t qts_full[2], qts_empty[2];
   uint64_t mma_done, mma_done2;
   uint32_t tmem_base;
   int abort_flag;
@@ -118,11 +124,16 @@ struct KParams {
 };
 
 // ------------------------------------------------------------ scheduling
+// Query tiles of user b from the cached query offsets.
+__device__ __forceinline__ int q_tiles(const int* mq, int b) {
+  return (mq[b + 1] - mq[b] + BM - 1) / BM;
+}
+
 __device__ __forceinline__ int count_users_above(const int* qt, int B, int lvl, int lane) {
   int c = 0;
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const bool p = b < B && qt[b] > lvl;
+    const bool p = b < B && q_tiles(qt, b) > lvl;
     c += __popc(__ballot_sync(0xffffffffu, p));
   }
   return c;
@@ -131,7 +142,7 @@ __device__ __forceinline__ int count_users_above(const int* qt, int B, int lvl, 
 __device__ __forceinline__ int nth_user_above(const int* qt, int B, int lvl, int n, int lane) {
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const bool p = b < B && qt[b] > lvl;
+    const bool p = b < B && q_tiles(qt, b) > lvl;
     unsigned m = __ballot_sync(0xffffffffu, p);
     const int c = __popc(m);
     if (n < c) {
@@ -153,7 +164,7 @@ struct Sched {
     B = B_;
     HS = HS_;
     int mx = 0;
-    for (int b = lane; b < B; b += 32) mx = max(mx, qt[b]);
+    for (int b = lane; b < B; b += 32) mx = max(mx, q_tiles(qt, b));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     lvl = mx - 1;
@@ -196,26 +207,22 @@ struct Item {
 };
 
 template <bool PAGED, bool CAND>
-__device__ __forceinline__ Item make_item(const KParams& P, int b, int m, int rem) {
+__device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem) {
   Item it;
   it.b = b;
   it.m = m;
   it.h = rem / P.n_split;
   it.s = rem % P.n_split;
-  const int64_t qs = P.q_off[b], nq = P.q_off[b + 1] - qs;
+  const int64_t qs = sm.m_q[b], nq = (int64_t)sm.m_q[b + 1] - qs;
   it.q_row0 = qs + (int64_t)BM * m;
   it.nvalid = (int)min64(BM, nq - (int64_t)BM * m);
+  it.n_k = sm.m_nk[b];
   if (PAGED) {
-    // an out-of-range user id has no cached tokens (and no page list is read)
-    const int64_t u = P.users[b];
-    const bool known = u >= 0 && u < P.max_users;
-    it.user = known ? u : 0;
-    it.n_k = known ? P.lengths[u] : 0;
+    it.user = sm.m_kv[b];
     it.kv_row0 = 0;
   } else {
     it.user = 0;
-    it.kv_row0 = P.kv_off[b];
-    it.n_k = P.kv_off[b + 1] - it.kv_row0;
+    it.kv_row0 = sm.m_kv[b];
   }
   int total;
   if (CAND) {
@@ -301,9 +308,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
 
   // ---- setup
-  for (int b = tid; b < P.B; b += kThreads) {
-    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
-    sm.qt[b] = (int)((nq + BM - 1) / BM);
+  for (int b = tid; b <= P.B; b += kThreads) {
+    sm.m_q[b] = (int)P.q_off[b];
+    if (b == P.B) continue;
+    if (PAGED) {
+      // an out-of-range user id has no cached tokens (and no page list is read)
+      const int64_t u = P.users[b];
+      const bool known = u >= 0 && u < P.max_users;
+      sm.m_kv[b] = known ? (int)u : 0;
+      sm.m_nk[b] = known ? (int)P.lengths[u] : 0;
+    } else {
+      sm.m_kv[b] = (int)P.kv_off[b];
+      sm.m_nk[b] = (int)(P.kv_off[b + 1] - P.kv_off[b]);
+    }
   }
   for (int i = tid; i < kMaxRab; i += kThreads) {
     sm.pos_ext[i] = P.pos_table ? P.pos_table[min(i, P.n_pos - 1)] : 0.f;
@@ -335,6 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.ts_full[i]), 1);
       mbar_init(smem_u32(&sm.ts_empty[i]), 8);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.qts_full[i]), 1);
+      mbar_init(smem_u32(&sm.qts_empty[i]), 16);
+    }
     mbar_init(smem_u32(&sm.mma_done), 1);
     mbar_init(smem_u32(&sm.mma_done2), 1);
     fence_mbar_init();
@@ -359,14 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // =============================================== TMA producer
     Sched sc;
-    sc.init(sm.qt, P.B, HS, lane);
+    sc.init(sm.m_q, P.B, HS, lane);
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
       const long long t = snake_item(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
         const uint32_t qs = qi % QST;
@@ -381,6 +402,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       ++qi;
+      if (PAGED) {
+        // page ids of this item's key tiles, staged once (coalesced) instead of
+        // one dependent global load per tile
+        const int32_t* plist = P.page_lists + it.user * (int64_t)P.max_ppu;
+        const int first = it.t0 * 4;
+        const int cnt = min((it.t1 - it.t0) * 4, kPagesStaged);
+        __syncwarp();
+        for (int i = lane; i < cnt; i += 32) {
+          const int idx = first + i;
+          sm.pages[i] = idx < P.max_ppu ? plist[idx] : -1;
+        }
+        __syncwarp();
+      }
       // Issue order K0, K1, V0, K2, V1, ... keeps K one tile ahead of V.
       const int nt = it.t1 - it.t0;
       for (int i = 0; i <= nt && ok; ++i) {
@@ -415,7 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int pg = 0; pg < 4; ++pg) {
                 const int idx = tile * 4 + pg;
-                int64_t page = idx < P.max_ppu ? (int64_t)plist[idx] : -1;
+                const int si = (tile - it.t0) * 4 + pg;
+                int64_t page = si < kPagesStaged ? (int64_t)sm.pages[si]
+                                                 : (idx < P.max_ppu ? (int64_t)plist[idx] : -1);
                 if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
                 const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
                 tma_load_2d(dst + pg * 4096, &tm_k, bar, 0, row);
@@ -454,15 +490,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
     // tensor pipe fed: while one waits on its barriers the other's MMAs run.
     Sched sc;
-    sc.init(sm.qt, P.B, HS, lane);
+    sc.init(sm.m_q, P.B, HS, lane);
     const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       const long long t = snake_item(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       const int nt = it.t1 - it.t0;
       if (lane == 0) {
@@ -531,16 +567,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // time-gap bias, so the pointwise warps never wait on global loads.
     if (P.time_table != nullptr && !PAGED && !CAND) {
       Sched sc;
-      sc.init(sm.qt, P.B, HS, lane);
-      uint32_t g = 0;
+      sc.init(sm.m_q, P.B, HS, lane);
+      uint32_t g = 0, qitem = 0;
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
       const long long t = snake_item(rnd);
         int b, m, rem;
-        if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
-        const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+        if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
+        const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
         if (it.t0 >= it.t1) continue;
         const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
+        {  // query timestamps of this item's rows
+          const uint32_t qsl = qitem & 1;
+          ok = mbar_wait_warp(smem_u32(&sm.qts_empty[qsl]), ((qitem >> 1) & 1) ^ 1);
+          if (!ok) break;
+          TsSlot& qs = sm.qts[qsl];
+          bool exact = true;
+#pragma unroll
+          for (int i = 0; i < BM / 32; ++i) {
+            const int r = lane + 32 * i;
+            long long v = base;
+            if (r < it.nvalid && it.n_k > 0) {
+              const int64_t qpc = min64(max64(it.p0 + r, 0), it.n_k - 1);
+              v = P.ts[it.kv_row0 + qpc];
+            }
+            const long long rel = v - base;
+            exact = exact && rel > -(1LL << 23) && rel < (1LL << 23);
+            qs.i[r] = v;
+            qs.f[r] = (float)rel;
+          }
+          exact = __all_sync(0xffffffffu, exact);
+          if (lane == 0) qs.exact = exact ? 1 : 0;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.qts_full[qsl]));
+          ++qitem;
+        }
         for (int tile = it.t0; tile < it.t1; ++tile, ++g) {
           const uint32_t slot = g % NTS;
           ok = mbar_wait_warp(smem_u32(&sm.ts_empty[slot]), ((g / NTS) & 1) ^ 1);
@@ -581,33 +642,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool use_pos = P.pos_table != nullptr;
     float* rrow = sm.rrow[pwi];
     Sched sc;
-    sc.init(sm.qt, P.B, HS, lane);
+    sc.init(sm.m_q, P.B, HS, lane);
     uint32_t qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       const long long t = snake_item(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.qt, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, b, m, rem);
+      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
       long long tq_i = 0;
       float tq1 = 1.f;
       bool tq_exact = true;
-      if (use_time && it.n_k > 0) {
-        const long long base = P.ts[it.kv_row0];
-        if (r < it.nvalid) {
-          const int64_t qpc = min64(max64(qp, 0), it.n_k - 1);
-          tq_i = P.ts[it.kv_row0 + qpc];
-        } else {
-          tq_i = base;
-        }
-        const long long rel = tq_i - base;
-        tq_exact = rel > -(1LL << 23) && rel < (1LL << 23);
-        tq1 = (float)rel + 1.f;
+      const uint32_t qsl = qi & 1;
+      if (use_time) {  // this row's timestamp, staged by warp 2
+        ok = mbar_wait_warp(smem_u32(&sm.qts_full[qsl]), (qi >> 1) & 1);
+        if (!ok) break;
+        tq_i = sm.qts[qsl].i[r];
+        tq1 = sm.qts[qsl].f[r] + 1.f;
+        tq_exact = sm.qts[qsl].exact != 0;
       }
-      tq_exact = __all_sync(0xffffffffu, tq_exact);
       for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
         if ((int)(g & 1) != wg) continue;
         const uint32_t sb = g & 1;
@@ -618,17 +674,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrel0 = __shfl_sync(0xffffffffu, qrel, 0);  // smallest in the warp
         const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
         // position-bias row of this warp: rrow[j] = pos bias at delta qrel0 + j - 127
+        // rrow[j] = position bias at delta qrel0 + j + roff - 127; this warp's
+        // columns need j in [0, 95) (roff = 64 for the low column half)
+        const int roff = chalf ? 0 : 64;
         if (use_pos && !cand_tile) {
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < RROW / 32; ++i) {
             const int j = lane + 32 * i;
-            const int delta = max(qrel0 + j - 127, 0);
+            const int delta = max(qrel0 + j + roff - 127, 0);
             rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
           }
           __syncwarp();
         }
-        const float* rl = use_pos ? (CAND ? rrow : rrow + lane) : sm.pos_ext;  // zeros without a table
+        // element (row lane, column c) reads rbase[127 - c]
+        const int rshift = use_pos ? ((CAND ? 0 : lane) - roff) : 0;
+        const float* rtab = use_pos ? rrow : sm.pos_ext;  // zeros without a table
         const uint32_t tslot = g % NTS;
         bool time_fast = false;
         if (use_time) {
@@ -672,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               cls = (cb + 31 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
               mk = 1;
             }
-            const float* rlc = rl + 127 - cb;
+            const float* rlc = rtab + (rshift + 127 - cb);
             if (cls == 2) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) pk[q][j] = 0u;
@@ -716,6 +777,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       }
       if (!ok) break;
+      if (use_time) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.qts_empty[qsl]));
+      }
       // ---- epilogue: this warpgroup stores O columns [ocol, ocol + 32)
       ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
       if (!ok) break;
@@ -885,8 +950,20 @@ size_t attn_sm100_workspace_bytes(const AttnProblem& p, int num_sms) {
 cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_bytes,
                               int* err_word, cudaStream_t stream) {
   if (p.d != HD || p.f32) return cudaErrorInvalidValue;
-  if (p.B > kMaxUsers) return cudaErrorInvalidValue;
   if (p.B == 0 || p.total_q == 0) return cudaSuccess;
+  if (p.B > kMaxUsers) {
+    // users are independent and offsets are absolute rows: run chunks of users
+    for (int b0 = 0; b0 < p.B; b0 += kMaxUsers) {
+      AttnProblem c = p;
+      c.B = std::min(kMaxUsers, p.B - b0);
+      c.q_off = p.q_off + b0;
+      if (p.kv_off) c.kv_off = p.kv_off + b0;
+      if (p.users) c.users = p.users + b0;
+      const cudaError_t e = attn_sm100_launch(c, workspace, ws_bytes, err_word, stream);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const int num_sms = device_sm_count();
   KParams kp;
   std::memset(&kp, 0, sizeof(kp));
