@@ -23,8 +23,9 @@
 //   warps 4-19  four "pointwise" warpgroups: two pairs alternate key tiles, the
 //               two warpgroups of a pair split the tile's 128 score columns;
 //               read S from TMEM, add the biases, mask, SiLU (via tanh), pack
-//               P to bf16 in TMEM; then the epilogue (O * scale -> bf16 or fp32
-//               split partial), 32 output columns per warpgroup.
+//               P to bf16 in TMEM; the pair that took an item's last key tile
+//               also runs its epilogue (O * scale -> bf16 or fp32 split partial)
+//               while the other pair starts the next item.
 // There is no softmax, so there is no running max and no rescaling of O, and
 // key splits of one query tile add exactly (the candidate path splits keys).
 // Work items (user, head, query tile, split) run longest-first: query tiles
@@ -70,8 +71,9 @@ constexpr int RROW = 96;            // position-bias row per pointwise warp (its
 struct TsSlot {
   float f[BN];
   long long i[BN];
-  int exact;
-  int pad[3];
+  int exact;     // every offset fits 23 bits (the float path is exact)
+  int sorted;    // key timestamps non-decreasing over the valid keys
+  int pad[2];
 };
 
 struct __align__(1024) Smem {
@@ -92,7 +94,7 @@ struct __align__(1024) Smem {
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
-  uint64_t o_full, o_empty;
+  uint64_t o_full[2], o_empty;   // o_full per pointwise pair (the pair that runs the epilogue)
   uint64_t ts_full[NTS], ts_empty[NTS];
   uint64_t qts_full[2], qts_empty[2];
   uint64_t mma_done, mma_done2;
@@ -346,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.p_full[i]), 8);
       mbar_init(smem_u32(&sm.p_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.o_empty), 16);
+    mbar_init(smem_u32(&sm.o_full[0]), 1);
+    mbar_init(smem_u32(&sm.o_full[1]), 1);
+    mbar_init(smem_u32(&sm.o_empty), 8);
     for (int i = 0; i < NTS; ++i) {
       mbar_init(smem_u32(&sm.ts_full[i]), 1);
       mbar_init(smem_u32(&sm.ts_empty[i]), 8);
@@ -546,7 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(smem_u32(&sm.v_empty[slot]));
             umma_commit(smem_u32(&sm.p_empty[pb]));
           }
-          if (ok) umma_commit(smem_u32(&sm.o_full));
+          // the pair that processed the item's last key tile runs its epilogue
+          if (ok) umma_commit(smem_u32(&sm.o_full[(g - 1) & 1]));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -597,7 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             qs.f[r] = (float)rel;
           }
           exact = __all_sync(0xffffffffu, exact);
-          if (lane == 0) qs.exact = exact ? 1 : 0;
+          if (lane == 0) {
+            qs.exact = exact ? 1 : 0;
+            qs.sorted = 0;
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.qts_full[qsl]));
           ++qitem;
@@ -620,7 +627,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ts.f[c] = (float)rel;
           }
           exact = __all_sync(0xffffffffu, exact);
-          if (lane == 0) ts.exact = exact ? 1 : 0;
+          __syncwarp();
+          bool sorted = true;
+#pragma unroll
+          for (int i = 0; i < BN / 32; ++i) {
+            const int c = lane + 32 * i;
+            const int64_t kp = (int64_t)tile * BN + c;
+            if (c + 1 < BN && kp + 1 < it.n_k) sorted = sorted && ts.i[c] <= ts.i[c + 1];
+          }
+          sorted = __all_sync(0xffffffffu, sorted);
+          if (lane == 0) {
+            ts.exact = exact ? 1 : 0;
+            ts.sorted = sorted ? 1 : 0;
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.ts_full[slot]));
         }
@@ -634,7 +653,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pwi = warp - 4;                       // 0..15
     const int wg = pwi >> 3;                        // tile parity handled
     const int chalf = (pwi >> 2) & 1;               // column half of the tile
-    const int ocol = (pwi >> 2) * 32;               // epilogue: O columns [ocol, ocol + 32)
     const int sub = warp & 3;                       // TMEM lane quarter
     const int r = sub * 32 + lane;                  // tile row owned by this thread
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
@@ -643,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* rrow = sm.rrow[pwi];
     Sched sc;
     sc.init(sm.m_q, P.B, HS, lane);
-    uint32_t qi = 0, g = 0;
+    uint32_t qi = 0, g = 0, my_epi = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       const long long t = snake_item(rnd);
@@ -703,6 +721,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_addr = tmem + lane_addr + TM_S0 + sb * 128;
         const uint32_t p_addr = tmem + lane_addr + TM_P0 + sb * 64;
         const float self_rab = sm.pos_ext[0];
+        // Far from the diagonal a row's 64 columns usually share one position
+        // bucket (and, with sorted key timestamps, one time bucket): then the
+        // whole bias is one constant per row and is folded into the SiLU.
+        float crow = 0.f;
+        bool rowconst = false;
+        if (!cand_tile) {
+          const int cbase = 64 * chalf;
+          const int dmax = qrel - cbase, dmin = qrel - cbase - 63;
+          bool ok_row = dmin >= 0 || CAND;  // every column of both chunks visible
+          if (CAND) ok_row = cbase + 63 < kend;
+          if (use_pos) {
+            const int b_hi = min(31 - __clz(max(dmax, 0) + 1), kMaxRab - 1);
+            const int b_lo = min(31 - __clz(max(dmin, 0) + 1), kMaxRab - 1);
+            ok_row = ok_row && sm.pos_ext[b_hi] == sm.pos_ext[b_lo];
+            crow = sm.pos_ext[b_hi];
+          }
+          if (use_time) {
+            const TsSlot& ts = sm.ts[tslot];
+            long long d_hi = tq_i - ts.i[cbase], d_lo = tq_i - ts.i[cbase + 63];
+            d_hi = d_hi < 0 ? 0 : d_hi;
+            d_lo = d_lo < 0 ? 0 : d_lo;
+            const int t_hi = min(63 - __clzll(d_hi + 1), kMaxRab - 1);
+            const int t_lo = min(63 - __clzll(d_lo + 1), kMaxRab - 1);
+            ok_row = ok_row && ts.sorted && sm.time_ext[t_hi] == sm.time_ext[t_lo];
+            crow += sm.time_ext[t_hi];
+          }
+          rowconst = __all_sync(0xffffffffu, ok_row);
+        }
+        const float hrow = 0.5f * crow;
         {
           const int half = chalf;
           uint32_t pk[2][16];
@@ -734,7 +781,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               mk = 1;
             }
             const float* rlc = rtab + (rshift + 127 - cb);
-            if (cls == 2) {
+            if (rowconst) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const float h0 = fmaf(0.5f, __uint_as_float(sv[j]), hrow);
+                const float h1 = fmaf(0.5f, __uint_as_float(sv[j + 1]), hrow);
+                pk[q][j >> 1] = pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
+              }
+            } else if (cls == 2) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) pk[q][j] = 0u;
             } else if (use_time) {
@@ -781,20 +835,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.qts_empty[qsl]));
       }
-      // ---- epilogue: this warpgroup stores O columns [ocol, ocol + 32)
-      ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
+      // ---- epilogue, by the pair that processed the item's last key tile (so
+      // the other pair can start the next item at once); this warp stores O
+      // columns [64 chalf, 64 chalf + 64) of its 32 rows.
+      if ((int)((g - 1) & 1) != wg) {
+        ++qi;
+        continue;
+      }
+      // each pair has its own o_full barrier and waits every one of its phases
+      // in order (a parity wait must never run two phases ahead or behind)
+      ok = mbar_wait_warp(smem_u32(&sm.o_full[wg]), my_epi & 1);
+      ++my_epi;
       if (!ok) break;
       tc_fence_after();
-      uint32_t oa[32];
-      tmem_ld32(tmem + lane_addr + TM_O + ocol, oa);
-      tmem_wait_ld();
-      reg_fence(oa);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
-      ++qi;
-      if (r < it.nvalid && it.q_row0 + r < P.total_q) {
-        const int64_t row = it.q_row0 + r;
+      const bool row_ok = r < it.nvalid && it.q_row0 + r < P.total_q;
+      const int64_t row = it.q_row0 + r;
+#pragma unroll 1
+      for (int q = 0; q < 2; ++q) {
+        const int ocol = 64 * chalf + 32 * q;
+        uint32_t oa[32];
+        tmem_ld32(tmem + lane_addr + TM_O + ocol, oa);
+        tmem_wait_ld();
+        reg_fence(oa);
+        if (q == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
+        }
+        if (!row_ok) continue;
         if (P.partial) {
           float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
                        it.h * HD + ocol;
@@ -817,6 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ++qi;
     }
     if (!ok && lane == 0) record_timeout(P, sm);
   }
@@ -916,8 +985,9 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, int grid, cudaS
   return cudaGetLastError();
 }
 
-// Key-split plan for the candidate path: enough (user, head, split) items to
-// cover the SMs about twice.
+// Key-split plan for the candidate path: one wave of (user, head, split)
+// items, each streaming a long run of key tiles (fewer pipeline start-ups and
+// fewer partial sums than many short splits).
 void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
   *n_split = 1;
   *kps = 1 << 30;
@@ -926,7 +996,7 @@ void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
   const int qt = std::max(1, (p.max_q + BM - 1) / BM);
   const long long base_items = (long long)p.B * p.H * qt;
   if (base_items <= 0) return;
-  int want = (int)std::min<long long>(max_tiles, (2LL * num_sms + base_items - 1) / base_items);
+  int want = (int)std::min<long long>(max_tiles, num_sms / base_items);
   if (want <= 1) return;
   int k = (max_tiles + want - 1) / want;
   k = std::max(k, 2);

@@ -59,15 +59,19 @@ def test_bf16_simt_head_dims(d):
 
 
 @pytest.mark.parametrize("lengths", [
+    [128] * 300,                # many one-tile users: item-to-item hand-offs
+    [256] * 64 + [1] * 7,       # two-tile users and single tokens
     [130, 300, 517],            # several tiles, ragged tails
     [1, 128, 129, 255, 256],    # tile-boundary edge cases
     [0, 7, 0, 384, 0],          # empty users
     [1000],
 ])
 def test_bf16_tcgen05_pos_rab(lengths):
+    # edge shapes: short users make scale = 1/max_len large, so outputs reach a few
+    # units and one bf16 ulp exceeds 1e-2 -> the ulp-aware elementwise bound
     case = workloads.jagged_case(7, lengths, H=4, d=128, dtype="bf16", n_pos=16)
     got, ref = run_case(case)
-    assert_bf16_close(got, ref, f"bf16 {lengths}")
+    assert_bf16_close(got, ref, f"bf16 {lengths[:8]}...", ulp_aware=True)
 
 
 def test_bf16_tcgen05_pos_time_rab():
