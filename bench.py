@@ -128,23 +128,13 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from generative_recommender_sequence_b200.sharding import global_step_time
+    return global_step_time(x, device="cuda") if world > 1 else x
 
 
 def sum_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    from generative_recommender_sequence_b200.sharding import global_units
+    return global_units(x, device="cuda") if world > 1 else x
 
 
 def _dev(a, dt=None):
@@ -249,8 +239,10 @@ def run_gpu(args):
     rank, world, local = dist_setup(args.gpus)
     hbm_peak, tf_peak, tf_sus, peak_src = load_peaks()
     n_total = args.warmup + args.steps + 12
-    A = PagedPart(W.long_history(), n_total, seed=55)
-    Bp = PagedPart(W.cached_cand(), n_total, seed=77)
+    # weak scaling: every rank owns one per-GPU batch of distinct users (its own
+    # seeds; rank 0 draws the reference workloads), no data-path collective
+    A = PagedPart(W.long_history(seed=1005 + 7919 * rank), n_total, seed=55 + rank)
+    Bp = PagedPart(W.cached_cand(seed=1003 + 7919 * rank), n_total, seed=77 + rank)
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -440,15 +432,15 @@ def run_oracle_sample(c5, rows5, c3, rows3, threads, kv5=None, kv3=None):
 def cpu_baseline(args):
     import oracle
     threads = oracle.default_threads()
-    c5, rows5, f5, c3, rows3, f3 = cpu_sample_units(rows_per_user=12, cands_per_user=4)
+    c5, rows5, f5, c3, rows3, f3 = cpu_sample_units(rows_per_user=300, cands_per_user=32)
     kv5, kv3 = _joined_kv(c5), _joined_kv(c3)
     t0 = time.perf_counter()
     run_oracle_sample(c5, rows5, c3, rows3, threads, kv5, kv3)
     dt = time.perf_counter() - t0
     return {"value": round((f5 + f3) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"fp64 C oracle on {len(rows5)} query rows of long_history (12 per user) + "
-                      f"{len(rows3)} candidates of cached_cand (4 per user); {dt:.1f} s"}
+            "sample": f"fp64 C oracle on {len(rows5)} query rows of long_history (up to 300 per user) + "
+                      f"{len(rows3)} candidates of cached_cand (32 per user); {dt:.1f} s"}
 
 
 def run_reference(args):
