@@ -257,15 +257,15 @@ __device__ __forceinline__ void record_timeout(const KParams& P, Smem& sm) {
 // 3 only the candidate's own key (c == r).  TIME: 0 none, 1 float-exponent
 // bucket (exact offsets), 2 int64 bucket.  rlc[-j] is the position bias of
 // column cb + j; tx is the time table with its clamp baked in (256 entries).
-template <int MASK, int TIME>
-__device__ __forceinline__ void pw_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16], const int cb,
+template <int MASK, int TIME, int W = 16>
+__device__ __forceinline__ void pw_chunk(const uint32_t (&sv)[W], uint32_t (&pk)[W / 2], const int cb,
                                          const float* __restrict__ rlc, const int qrel,
                                          const int kend, const int r, const float* ktf,
                                          const long long* kti, const float tq1,
                                          const long long tqi, const float* tx,
                                          const float self_rab) {
 #pragma unroll
-  for (int j = 0; j < 32; j += 4) {
+  for (int j = 0; j < W; j += 4) {
     float4 kt4;
     if (TIME == 1) kt4 = *reinterpret_cast<const float4*>(ktf + cb + j);
     float pv[4];
@@ -752,45 +752,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float hrow = 0.5f * crow;
         {
           const int half = chalf;
-          uint32_t pk[2][16];
+          uint32_t pk[4][8];
+          uint32_t sbuf[2][16];
+          tmem_ld16(s_addr + half * 64, sbuf[0]);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int cb = half * 64 + q * 32;
-            uint32_t sv[32];
-            tmem_ld32(s_addr + cb, sv);
+          for (int q = 0; q < 4; ++q) {
+            const int cb = half * 64 + q * 16;
+            // wait for chunk q, then start loading chunk q + 1 before computing q
             tmem_wait_ld();
-            reg_fence(sv);
-            if (q == 1) {  // this warp's part of S is in registers: the buffer may be rewritten
+            reg_fence(sbuf[q & 1]);
+            if (q < 3) {
+              tmem_ld16(s_addr + cb + 16, sbuf[(q + 1) & 1]);
+            } else {  // all of this warp's S is in registers: the buffer may be rewritten
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
             }
-            // warp-uniform mask class of this 32-column chunk
+            const uint32_t (&sv)[16] = sbuf[q & 1];
+            // warp-uniform mask class of this 16-column chunk
             int cls;  // 0 visible, 1 per-element, 2 none visible
             int mk;   // per-element mask kind
             if (CAND) {
               if (cand_tile) {
-                cls = (cb == 32 * sub) ? 1 : 2;
+                cls = (cb >> 5) == sub ? 1 : 2;
                 mk = 3;
               } else {
-                cls = (cb + 31 < kend) ? 0 : (cb >= kend ? 2 : 1);
+                cls = (cb + 15 < kend) ? 0 : (cb >= kend ? 2 : 1);
                 mk = 2;
               }
             } else {
-              cls = (cb + 31 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
+              cls = (cb + 15 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
               mk = 1;
             }
             const float* rlc = rtab + (rshift + 127 - cb);
             if (rowconst) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 2) {
+              for (int j = 0; j < 16; j += 2) {
                 const float h0 = fmaf(0.5f, __uint_as_float(sv[j]), hrow);
                 const float h1 = fmaf(0.5f, __uint_as_float(sv[j + 1]), hrow);
                 pk[q][j >> 1] = pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
               }
             } else if (cls == 2) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) pk[q][j] = 0u;
+              for (int j = 0; j < 8; ++j) pk[q][j] = 0u;
             } else if (use_time) {
               const TsSlot& ts = sm.ts[tslot];
               if (time_fast) {
@@ -821,8 +825,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
           if (!ok) break;
           tc_fence_after();
-          tmem_st16(p_addr + half * 32, pk[0]);
-          tmem_st16(p_addr + half * 32 + 16, pk[1]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_st8(p_addr + half * 32 + q * 8, pk[q]);
         }
         if (!ok) break;
         tmem_wait_st();
