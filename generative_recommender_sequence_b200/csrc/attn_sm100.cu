@@ -17,8 +17,9 @@
 //   warp 0      TMA producer: Q tile (128 x 128), K ring (2 x 128 x 128), Q double buffer,
 //               V ring (2 x 128 x 128), all 128-byte swizzled.  Paged keys are
 //               four 32-token page boxes per 128-key tile.
-//   warp 1      tcgen05 issuer of S = Q K^T into TMEM (two S buffers)
-//   warp 3      tcgen05 issuer of O += P V, P read from TMEM (two bf16 P buffers)
+//   warp 1      tcgen05 issuer of S = Q K^T into TMEM (three S/P buffers)
+//   warp 3      tcgen05 issuer of O += P V, P read from TMEM (bf16 P written over
+//               the start of each warpgroup's S columns)
 //   warp 2      stages key timestamps for the time-gap bias (mbarrier ring)
 //   warps 4-19  four "pointwise" warpgroups: two pairs alternate key tiles, the
 //               two warpgroups of a pair split the tile's 128 score columns;
@@ -56,7 +57,12 @@ constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 12
 constexpr int kMaxUsers = 1024;   // per launch; larger batches are split on the host
 constexpr int kMaxRab = 256;
 
-constexpr uint32_t TM_O = 0, TM_S0 = 128, TM_P0 = 384;  // S1 = S0 + 128, P1 = P0 + 64
+constexpr uint32_t TM_O = 0;      // O accumulator, 128 fp32 columns
+constexpr uint32_t TM_SP = 128;    // three S/P buffers of 128 columns each
+constexpr int NSP = 3;
+// P (bf16 pairs) overwrites the start of each warpgroup's own S columns:
+// keys 0-63 -> columns 0-31, keys 64-127 -> columns 64-95 of the buffer.
+__host__ __device__ constexpr uint32_t p_col(int kk) { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; }
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
@@ -92,8 +98,9 @@ struct __align__(1024) Smem {
   uint64_t q_full[QST], q_empty[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
+  // s_full per (pair, buffer) = tile index mod 6, so each pair waits every phase
+  // of its own barriers in order; p_full / sp_empty have one in-order waiter
+  uint64_t s_full[2 * NSP], p_full[NSP], sp_empty[NSP];
   uint64_t o_full[2], o_empty;   // o_full per pointwise pair (the pair that runs the epilogue)
   uint64_t ts_full[NTS], ts_empty[NTS];
   uint64_t qts_full[2], qts_empty[2];
@@ -342,11 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.v_full[i]), 1);
       mbar_init(smem_u32(&sm.v_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_empty[i]), 8);
+    for (int i = 0; i < 2 * NSP; ++i) mbar_init(smem_u32(&sm.s_full[i]), 1);
+    for (int i = 0; i < NSP; ++i) {
       mbar_init(smem_u32(&sm.p_full[i]), 8);
-      mbar_init(smem_u32(&sm.p_empty[i]), 1);
+      mbar_init(smem_u32(&sm.sp_empty[i]), 1);
     }
     mbar_init(smem_u32(&sm.o_full[0]), 1);
     mbar_init(smem_u32(&sm.o_full[1]), 1);
@@ -510,9 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t q_base = smem_u32(sm.q[qs]);
           ok = mbar_wait(smem_u32(&sm.q_full[qs]), (qi / QST) & 1);
           for (int i = 0; i < nt && ok; ++i, ++g, ++kc) {
-            const uint32_t sb = g & 1;
+            const uint32_t sb = g % NSP;
             const uint32_t slot = kc % KST;
-            ok = mbar_wait(smem_u32(&sm.s_empty[sb]), ((g >> 1) & 1) ^ 1) &&
+            // the buffer is free once the O += P V that read its P completed
+            ok = mbar_wait(smem_u32(&sm.sp_empty[sb]), ((g / NSP) & 1) ^ 1) &&
                  mbar_wait(smem_u32(&sm.k_full[slot]), (kc / KST) & 1);
             if (!ok) break;
             tc_fence_after();
@@ -522,17 +529,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
               const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
               const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-              umma_ss(tmem + TM_S0 + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+              umma_ss(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
             }
             umma_commit(smem_u32(&sm.k_empty[slot]));
-            umma_commit(smem_u32(&sm.s_full[sb]));
+            umma_commit(smem_u32(&sm.s_full[g % (2 * NSP)]));
             if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
           }
         } else {
           for (int i = 0; i < nt && ok; ++i, ++g, ++vc) {
-            const uint32_t pb = g & 1;
+            const uint32_t pb = g % NSP;
             const uint32_t slot = vc % VST;
-            ok = mbar_wait(smem_u32(&sm.p_full[pb]), (g >> 1) & 1) &&
+            ok = mbar_wait(smem_u32(&sm.p_full[pb]), (g / NSP) & 1) &&
                  mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1) &&
                  (i != 0 || mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
             if (!ok) break;
@@ -543,11 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key
               // groups 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
               const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
-              umma_ts(tmem + TM_O, tmem + TM_P0 + pb * 64 + kk * 8, bdesc, kIdescPV,
+              umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV,
                       (i == 0 && kk == 0) ? 0u : 1u);
             }
             umma_commit(smem_u32(&sm.v_empty[slot]));
-            umma_commit(smem_u32(&sm.p_empty[pb]));
+            umma_commit(smem_u32(&sm.sp_empty[pb]));
           }
           // the pair that processed the item's last key tile runs its epilogue
           if (ok) umma_commit(smem_u32(&sm.o_full[(g - 1) & 1]));
@@ -684,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
         if ((int)(g & 1) != wg) continue;
-        const uint32_t sb = g & 1;
+        const uint32_t sb = g % NSP;
         const bool cand_tile = CAND && tile == it.n_main;
         const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
         // int32 tile-relative coordinates: query position minus k0, valid keys
@@ -715,11 +722,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           time_fast = tq_exact && sm.ts[tslot].exact;
         }
-        ok = mbar_wait_warp(smem_u32(&sm.s_full[sb]), (g >> 1) & 1);
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_addr + TM_S0 + sb * 128;
-        const uint32_t p_addr = tmem + lane_addr + TM_P0 + sb * 64;
+        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128;
+        // P of this warpgroup's 64 keys overwrites the start of its own S columns
+        const uint32_t p_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
         const float self_rab = sm.pos_ext[0];
         // Far from the diagonal a row's 64 columns usually share one position
         // bucket (and, with sorted key timestamps, one time bucket): then the
@@ -761,13 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // wait for chunk q, then start loading chunk q + 1 before computing q
             tmem_wait_ld();
             reg_fence(sbuf[q & 1]);
-            if (q < 3) {
-              tmem_ld16(s_addr + cb + 16, sbuf[(q + 1) & 1]);
-            } else {  // all of this warp's S is in registers: the buffer may be rewritten
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
-            }
+            if (q < 3) tmem_ld16(s_addr + cb + 16, sbuf[(q + 1) & 1]);
             const uint32_t (&sv)[16] = sbuf[q & 1];
             // warp-uniform mask class of this 16-column chunk
             int cls;  // 0 visible, 1 per-element, 2 none visible
@@ -822,11 +824,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
           }
-          ok = mbar_wait_warp(smem_u32(&sm.p_empty[sb]), ((g >> 1) & 1) ^ 1);
-          if (!ok) break;
-          tc_fence_after();
+          // every S column of this warp is in registers (the last load was
+          // waited for), so P may overwrite them
 #pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_st8(p_addr + half * 32 + q * 8, pk[q]);
+          for (int q = 0; q < 4; ++q) tmem_st8(p_addr + q * 8, pk[q]);
         }
         if (!ok) break;
         tmem_wait_st();
