@@ -424,57 +424,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      // Issue order K0, K1, V0, K2, V1, ... keeps K one tile ahead of V.
+      // Issue order K0, K1, V0, K2, V1, ... keeps K one tile ahead of V.  Lane 0
+      // waits for the slot and posts the byte count; the tile's boxes (two
+      // 64-column halves, times four pages when paged) are then issued by one
+      // lane each so that the per-copy issue cost is paid in parallel.
       const int nt = it.t1 - it.t0;
       for (int i = 0; i <= nt && ok; ++i) {
-        if (lane == 0) {
-          for (int which = 0; which < 2 && ok; ++which) {
-            // which == 0: K of tile i ; which == 1: V of tile i-1
-            const int ti = which == 0 ? i : i - 1;
-            if (ti < 0 || ti >= nt) continue;
-            const int tile = it.t0 + ti;
-            uint32_t slot, bar, dst;
-            if (which == 0) {
-              slot = kc % KST;
-              ok = mbar_wait(smem_u32(&sm.k_empty[slot]), ((kc / KST) & 1) ^ 1);
-              bar = smem_u32(&sm.k_full[slot]);
-              dst = smem_u32(sm.k[slot]);
-              ++kc;
-            } else {
-              slot = vc % VST;
-              ok = mbar_wait(smem_u32(&sm.v_empty[slot]), ((vc / VST) & 1) ^ 1);
-              bar = smem_u32(&sm.v_full[slot]);
-              dst = smem_u32(sm.v[slot]);
-              ++vc;
-            }
-            if (!ok) break;
-            mbar_arrive_expect_tx(bar, kTileBytes);
-            if (CAND && tile == it.n_main) {
-              const CUtensorMap* tm = which == 0 ? &tm_kc : &tm_vc;
-              tma_load_3d(dst, tm, bar, 0, it.h, (int)it.q_row0);
-              tma_load_3d(dst + kHalfBytes, tm, bar, 64, it.h, (int)it.q_row0);
-            } else if (PAGED) {
+        for (int which = 0; which < 2; ++which) {
+          // which == 0: K of tile i ; which == 1: V of tile i-1
+          const int ti = which == 0 ? i : i - 1;
+          if (ti < 0 || ti >= nt) continue;
+          const int tile = it.t0 + ti;
+          const uint32_t c = which == 0 ? kc : vc;
+          const uint32_t slot = which == 0 ? c % KST : c % VST;
+          const uint32_t par = (which == 0 ? (c / KST) & 1 : (c / VST) & 1) ^ 1;
+          const uint32_t bar = smem_u32(which == 0 ? &sm.k_full[slot] : &sm.v_full[slot]);
+          const uint32_t dst = smem_u32(which == 0 ? sm.k[slot] : sm.v[slot]);
+          if (lane == 0) {
+            ok = mbar_wait(smem_u32(which == 0 ? &sm.k_empty[slot] : &sm.v_empty[slot]), par);
+            if (ok) mbar_arrive_expect_tx(bar, kTileBytes);
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          if (which == 0) ++kc; else ++vc;
+          const int half = lane & 1;
+          if (CAND && tile == it.n_main) {
+            if (lane < 2)
+              tma_load_3d(dst + half * kHalfBytes, which == 0 ? &tm_kc : &tm_vc, bar, half * 64,
+                          it.h, (int)it.q_row0);
+          } else if (PAGED) {
+            if (lane < 8) {
+              const int pg = lane >> 1;
+              const int idx = tile * 4 + pg;
+              const int si = (tile - it.t0) * 4 + pg;
               const int32_t* plist = P.page_lists + it.user * (int64_t)P.max_ppu;
-#pragma unroll
-              for (int pg = 0; pg < 4; ++pg) {
-                const int idx = tile * 4 + pg;
-                const int si = (tile - it.t0) * 4 + pg;
-                int64_t page = si < kPagesStaged ? (int64_t)sm.pages[si]
-                                                 : (idx < P.max_ppu ? (int64_t)plist[idx] : -1);
-                if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
-                const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
-                tma_load_2d(dst + pg * 4096, &tm_k, bar, 0, row);
-                tma_load_2d(dst + kHalfBytes + pg * 4096, &tm_k, bar, 64, row);
-              }
-            } else {
-              const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
-              const int row = (int)(it.kv_row0 + (int64_t)tile * BN);
-              tma_load_3d(dst, tm, bar, 0, it.h, row);
-              tma_load_3d(dst + kHalfBytes, tm, bar, 64, it.h, row);
+              int64_t page = si < kPagesStaged ? (int64_t)sm.pages[si]
+                                               : (idx < P.max_ppu ? (int64_t)plist[idx] : -1);
+              if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
+              const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
+              tma_load_2d(dst + half * kHalfBytes + pg * 4096, &tm_k, bar, half * 64, row);
             }
+          } else if (lane < 2) {
+            const int row = (int)(it.kv_row0 + (int64_t)tile * BN);
+            tma_load_3d(dst + half * kHalfBytes, which == 0 ? &tm_k : &tm_v, bar, half * 64, it.h,
+                        row);
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
       if (!ok) break;
     }
