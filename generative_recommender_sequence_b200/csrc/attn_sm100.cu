@@ -302,6 +302,67 @@ __device__ __forceinline__ void pw_chunk(const uint32_t (&sv)[W], uint32_t (&pk)
   }
 }
 
+// SiLU of a 16-column chunk whose bias is one constant per row: with
+// h = (s + c) / 2, SiLU(s + c) = h + h tanh(h); hrow = c / 2.
+__device__ __forceinline__ void silu_rowconst(const uint32_t (&sv)[16], uint32_t (&pk)[8],
+                                              const float hrow) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float h0 = fmaf(0.5f, __uint_as_float(sv[j]), hrow);
+    const float h1 = fmaf(0.5f, __uint_as_float(sv[j + 1]), hrow);
+    pk[j >> 1] = pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
+  }
+}
+
+// One 16-column chunk off the constant-row path: picks the mask class of the
+// chunk (warp-uniform) and the bias form, then runs the matching pw_chunk.
+// tmode: 0 no time bias, 1 float-exponent buckets, 2 integer buckets.
+template <bool CAND>
+__device__ __forceinline__ void pw_chunk_any(const uint32_t (&sv)[16], uint32_t (&pk)[8],
+                                             const int cb, const bool cand_tile, const int sub,
+                                             const int qrel0, const int kend, const int tmode,
+                                             const float* rlc, const int qrel, const int r,
+                                             const TsSlot& ts, const float tq1,
+                                             const long long tq_i, const float* tx,
+                                             const float self_rab) {
+  int cls;  // 0 visible, 1 per-element, 2 none visible
+  int mk;   // per-element mask kind
+  if (CAND) {
+    if (cand_tile) {
+      cls = (cb >> 5) == sub ? 1 : 2;
+      mk = 3;
+    } else {
+      cls = (cb + 15 < kend) ? 0 : (cb >= kend ? 2 : 1);
+      mk = 2;
+    }
+  } else {
+    cls = (cb + 15 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
+    mk = 1;
+  }
+  if (cls == 2) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pk[j] = 0u;
+  } else if (!CAND && tmode == 1) {
+    if (cls == 0)
+      pw_chunk<0, 1>(sv, pk, cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, tx, self_rab);
+    else
+      pw_chunk<1, 1>(sv, pk, cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, tx, self_rab);
+  } else if (!CAND && tmode == 2) {
+    if (cls == 0)
+      pw_chunk<0, 2>(sv, pk, cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, tx, self_rab);
+    else
+      pw_chunk<1, 2>(sv, pk, cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, tx, self_rab);
+  } else if (cls == 0) {
+    pw_chunk<0, 0>(sv, pk, cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+  } else if (mk == 1) {
+    pw_chunk<1, 0>(sv, pk, cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+  } else if (mk == 2) {
+    pw_chunk<2, 0>(sv, pk, cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+  } else {
+    pw_chunk<3, 0>(sv, pk, cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
+  }
+}
+
 // ------------------------------------------------------------ the kernel
 template <bool PAGED, bool CAND>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -661,6 +722,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
     const bool use_pos = P.pos_table != nullptr;
     float* rrow = sm.rrow[pwi];
+    const float self_rab = sm.pos_ext[0];
+    // last position bucket this thread read, and its bias (tiles far from the
+    // diagonal keep the same bucket for long runs, so the shared table is
+    // rarely touched on the constant-row path)
+    int pb_idx = -1;
+    float pb_val = 0.f;
     Sched sc;
     sc.init(sm.m_q, P.B, HS, lane);
     uint32_t qi = 0, g = 0, my_epi = 0;
@@ -691,22 +758,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
         // int32 tile-relative coordinates: query position minus k0, valid keys
         const int qrel = (int)max64(min64(qp - k0, 1 << 30), -(1 << 30));
-        const int qrel0 = __shfl_sync(0xffffffffu, qrel, 0);  // smallest in the warp
+        // lane 0 has the warp's smallest query position
+        const int64_t qp0 = CAND ? it.p0 : it.p0 + sub * 32;
+        const int qrel0 = (int)max64(min64(qp0 - k0, 1 << 30), -(1 << 30));
         const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
-        // position-bias row of this warp: rrow[j] = pos bias at delta qrel0 + j - 127
-        // rrow[j] = position bias at delta qrel0 + j + roff - 127; this warp's
-        // columns need j in [0, 95) (roff = 64 for the low column half)
+        // offset of this warp's column half in its position-bias row
         const int roff = chalf ? 0 : 64;
-        if (use_pos && !cand_tile) {
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < RROW / 32; ++i) {
-            const int j = lane + 32 * i;
-            const int delta = max(qrel0 + j + roff - 127, 0);
-            rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
-          }
-          __syncwarp();
-        }
         // element (row lane, column c) reads rbase[127 - c]
         const int rshift = use_pos ? ((CAND ? 0 : lane) - roff) : 0;
         const float* rtab = use_pos ? rrow : sm.pos_ext;  // zeros without a table
@@ -717,13 +774,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           time_fast = tq_exact && sm.ts[tslot].exact;
         }
-        ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128;
-        // P of this warpgroup's 64 keys overwrites the start of its own S columns
-        const uint32_t p_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
-        const float self_rab = sm.pos_ext[0];
         // Far from the diagonal a row's 64 columns usually share one position
         // bucket (and, with sorted key timestamps, one time bucket): then the
         // whole bias is one constant per row and is folded into the SiLU.
@@ -737,8 +787,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use_pos) {
             const int b_hi = min(31 - __clz(max(dmax, 0) + 1), kMaxRab - 1);
             const int b_lo = min(31 - __clz(max(dmin, 0) + 1), kMaxRab - 1);
-            ok_row = ok_row && sm.pos_ext[b_hi] == sm.pos_ext[b_lo];
-            crow = sm.pos_ext[b_hi];
+            if (b_hi != pb_idx) {
+              pb_idx = b_hi;
+              pb_val = sm.pos_ext[b_hi];
+            }
+            ok_row = ok_row && (b_hi == b_lo || pb_val == sm.pos_ext[b_lo]);
+            crow = pb_val;
           }
           if (use_time) {
             const TsSlot& ts = sm.ts[tslot];
@@ -752,77 +806,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           rowconst = __all_sync(0xffffffffu, ok_row);
         }
+        // position-bias row of this warp, only needed off the constant-row path:
+        // rrow[j] = position bias at delta qrel0 + j + roff - 127; this warp's
+        // columns need j in [0, 95)
+        if (use_pos && !cand_tile && !rowconst) {
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < RROW / 32; ++i) {
+            const int j = lane + 32 * i;
+            const int delta = max(qrel0 + j + roff - 127, 0);
+            rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
+          }
+          __syncwarp();
+        }
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // this warp's 64 S columns and, over their first half, its 32 P columns
+        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
+        const uint32_t p_addr = s_addr;
         const float hrow = 0.5f * crow;
-        {
-          const int half = chalf;
-          uint32_t pk[4][8];
-          uint32_t sbuf[2][16];
-          tmem_ld16(s_addr + half * 64, sbuf[0]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int cb = half * 64 + q * 16;
-            // wait for chunk q, then start loading chunk q + 1 before computing q
+        // Two 16-column chunks per (rolled) iteration: chunk q + 1 loads while
+        // chunk q computes.  P of chunk q goes to columns [8q, 8q + 8), which
+        // only covers S chunks already loaded into registers.
+        uint32_t sa[16], sb2[16], pk[8];
+        tmem_ld16(s_addr, sa);
+        if (rowconst) {
+#pragma unroll 1
+          for (int q = 0; q < 4; q += 2) {
             tmem_wait_ld();
-            reg_fence(sbuf[q & 1]);
-            if (q < 3) tmem_ld16(s_addr + cb + 16, sbuf[(q + 1) & 1]);
-            const uint32_t (&sv)[16] = sbuf[q & 1];
-            // warp-uniform mask class of this 16-column chunk
-            int cls;  // 0 visible, 1 per-element, 2 none visible
-            int mk;   // per-element mask kind
-            if (CAND) {
-              if (cand_tile) {
-                cls = (cb >> 5) == sub ? 1 : 2;
-                mk = 3;
-              } else {
-                cls = (cb + 15 < kend) ? 0 : (cb >= kend ? 2 : 1);
-                mk = 2;
-              }
-            } else {
-              cls = (cb + 15 <= qrel0) ? 0 : (cb > qrel0 + 31 ? 2 : 1);
-              mk = 1;
-            }
-            const float* rlc = rtab + (rshift + 127 - cb);
-            if (rowconst) {
-#pragma unroll
-              for (int j = 0; j < 16; j += 2) {
-                const float h0 = fmaf(0.5f, __uint_as_float(sv[j]), hrow);
-                const float h1 = fmaf(0.5f, __uint_as_float(sv[j + 1]), hrow);
-                pk[q][j >> 1] = pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
-              }
-            } else if (cls == 2) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) pk[q][j] = 0u;
-            } else if (use_time) {
-              const TsSlot& ts = sm.ts[tslot];
-              if (time_fast) {
-                if (cls == 0)
-                  pw_chunk<0, 1>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
-                else
-                  pw_chunk<1, 1>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
-              } else {
-                if (cls == 0)
-                  pw_chunk<0, 2>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
-                else
-                  pw_chunk<1, 2>(sv, pk[q], cb, rlc, qrel, kend, r, ts.f, ts.i, tq1, tq_i, sm.time_ext, self_rab);
-              }
-            } else if (cls == 0) {
-              pw_chunk<0, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
-            } else if (mk == 1) {
-              pw_chunk<1, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
-            } else if (mk == 2) {
-              pw_chunk<2, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
-            } else {
-              pw_chunk<3, 0>(sv, pk[q], cb, rlc, qrel, kend, r, nullptr, nullptr, 0.f, 0, nullptr, self_rab);
-            }
+            reg_fence(sa);
+            tmem_ld16(s_addr + (q + 1) * 16, sb2);
+            silu_rowconst(sa, pk, hrow);
+            tmem_st8(p_addr + q * 8, pk);
+            tmem_wait_ld();
+            reg_fence(sb2);
+            if (q == 0) tmem_ld16(s_addr + 32, sa);
+            silu_rowconst(sb2, pk, hrow);
+            tmem_st8(p_addr + (q + 1) * 8, pk);
           }
-          if (use_time) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
+        } else {
+          const int cb0 = chalf * 64;
+          const float* rl0 = rtab + (rshift + 127 - cb0);
+          const TsSlot& ts = sm.ts[use_time ? tslot : 0];
+          const int tmode = use_time ? (time_fast ? 1 : 2) : 0;
+#pragma unroll 1
+          for (int q = 0; q < 4; q += 2) {
+            tmem_wait_ld();
+            reg_fence(sa);
+            tmem_ld16(s_addr + (q + 1) * 16, sb2);
+            pw_chunk_any<CAND>(sa, pk, cb0 + q * 16, cand_tile, sub, qrel0, kend, tmode, rl0 - q * 16,
+                               qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
+            tmem_st8(p_addr + q * 8, pk);
+            tmem_wait_ld();
+            reg_fence(sb2);
+            if (q == 0) tmem_ld16(s_addr + 32, sa);
+            pw_chunk_any<CAND>(sb2, pk, cb0 + q * 16 + 16, cand_tile, sub, qrel0, kend, tmode,
+                               rl0 - q * 16 - 16, qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
+            tmem_st8(p_addr + (q + 1) * 8, pk);
           }
-          // every S column of this warp is in registers (the last load was
-          // waited for), so P may overwrite them
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_st8(p_addr + q * 8, pk[q]);
+        }
+        if (use_time) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
         }
         if (!ok) break;
         tmem_wait_st();
