@@ -37,6 +37,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "attn.h"
@@ -54,22 +55,29 @@ constexpr int VST = 2;             // V ring depth
 constexpr int kThreads = 640;      // 20 warps: TMA, MMA, timestamps, spare, 16 pointwise
 constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
+constexpr int kPairHalfK = kHalfBytes / 2;  // CTA pair: one 64-column half of 64 keys
 constexpr int kMaxUsers = 1024;   // per launch; larger batches are split on the host
 constexpr int kMaxRab = 256;
 
 constexpr uint32_t TM_O = 0;      // O accumulator, 128 fp32 columns
 constexpr uint32_t TM_SP = 128;    // three S/P buffers of 128 columns each
 constexpr int NSP = 3;
-// P (bf16 pairs) overwrites the start of each warpgroup's own S columns:
-// keys 0-63 -> columns 0-31, keys 64-127 -> columns 64-95 of the buffer.
-__host__ __device__ constexpr uint32_t p_col(int kk) { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; }
+// whether eligible launches use CTA pairs when HSTU_ATTN_CTA_PAIRS is unset
+constexpr bool kCtaPairsByDefault = false;
+// P (bf16 pairs) overwrites the first half of each pointwise warp's own 32 S
+// columns: keys [32 c, 32 c + 32) -> columns [32 c, 32 c + 16) of the buffer,
+// so the 16 keys of MMA k-step kk start at column 32 (kk / 2) + 8 (kk % 2).
+__host__ __device__ constexpr uint32_t p_col(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
+// CTA pair: M = 256 rows over the two CTAs, each supplying half of B's N columns
+constexpr uint32_t kIdescQK2 = idesc_bf16_f32(2 * BM, BN, false);
+constexpr uint32_t kIdescPV2 = idesc_bf16_f32(2 * BM, HD, true);
 
 constexpr int NTS = 4;              // key-timestamp ring depth
 constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
-constexpr int RROW = 96;            // position-bias row per pointwise warp (its 64 columns + 31)
+constexpr int RROW = 64;            // position-bias row per pointwise warp (its 32 columns + 31)
 
 // Key timestamps of one key tile, staged by warp 2: exact float offsets from
 // the user's first timestamp (when |offset| < 2^23 for every key), plus the
@@ -100,8 +108,8 @@ struct __align__(1024) Smem {
   uint64_t v_full[VST], v_empty[VST];
   // s_full per (pair, buffer) = tile index mod 6, so each pair waits every phase
   // of its own barriers in order; p_full / sp_empty have one in-order waiter
-  uint64_t s_full[2 * NSP], p_full[NSP], sp_empty[NSP];
-  uint64_t o_full[2], o_empty;   // o_full per pointwise pair (the pair that runs the epilogue)
+  uint64_t s_full[NSP], p_full[NSP], sp_empty[NSP];
+  uint64_t o_full, o_empty;
   uint64_t ts_full[NTS], ts_empty[NTS];
   uint64_t qts_full[2], qts_empty[2];
   uint64_t mma_done, mma_done2;
@@ -133,25 +141,25 @@ struct KParams {
 };
 
 // ------------------------------------------------------------ scheduling
-// Query tiles of user b from the cached query offsets.
-__device__ __forceinline__ int q_tiles(const int* mq, int b) {
-  return (mq[b + 1] - mq[b] + BM - 1) / BM;
+// Query row blocks of user b (bm rows each) from the cached query offsets.
+__device__ __forceinline__ int q_tiles(const int* mq, int b, int bm) {
+  return (mq[b + 1] - mq[b] + bm - 1) / bm;
 }
 
-__device__ __forceinline__ int count_users_above(const int* qt, int B, int lvl, int lane) {
+__device__ __forceinline__ int count_users_above(const int* qt, int B, int lvl, int bm, int lane) {
   int c = 0;
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const bool p = b < B && q_tiles(qt, b) > lvl;
+    const bool p = b < B && q_tiles(qt, b, bm) > lvl;
     c += __popc(__ballot_sync(0xffffffffu, p));
   }
   return c;
 }
 
-__device__ __forceinline__ int nth_user_above(const int* qt, int B, int lvl, int n, int lane) {
+__device__ __forceinline__ int nth_user_above(const int* qt, int B, int lvl, int bm, int n, int lane) {
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const bool p = b < B && q_tiles(qt, b) > lvl;
+    const bool p = b < B && q_tiles(qt, b, bm) > lvl;
     unsigned m = __ballot_sync(0xffffffffu, p);
     const int c = __popc(m);
     if (n < c) {
@@ -165,6 +173,7 @@ __device__ __forceinline__ int nth_user_above(const int* qt, int B, int lvl, int
 
 // Item order: query-tile level from the highest down; within a level, users in
 // order, then heads, then key splits.  Warp-collective (all lanes agree).
+template <int bm>
 struct Sched {
   int lvl;
   long long base, cnt;
@@ -173,34 +182,37 @@ struct Sched {
     B = B_;
     HS = HS_;
     int mx = 0;
-    for (int b = lane; b < B; b += 32) mx = max(mx, q_tiles(qt, b));
+    for (int b = lane; b < B; b += 32) mx = max(mx, q_tiles(qt, b, bm));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     lvl = mx - 1;
     base = 0;
-    cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, lane) * HS : 0;
+    cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, bm, lane) * HS : 0;
   }
   __device__ bool item(long long t, const int* qt, int lane, int& b, int& m, int& rem) {
     while (lvl >= 0 && t >= base + cnt) {
       base += cnt;
       --lvl;
-      cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, lane) * HS : 0;
+      cnt = lvl >= 0 ? (long long)count_users_above(qt, B, lvl, bm, lane) * HS : 0;
     }
     if (lvl < 0) return false;
     const long long r = t - base;
     rem = (int)(r % HS);
-    b = nth_user_above(qt, B, lvl, (int)(r / HS), lane);
+    b = nth_user_above(qt, B, lvl, bm, (int)(r / HS), lane);
     m = lvl;
     return b >= 0;
   }
 };
 
-// Items are sorted longest first; round k hands them to the CTAs in forward
-// order for even k and in reverse order for odd k (a snake), so the CTA that
-// got the longest item of one round gets the shortest of the next.
+// Items are sorted longest first; round k hands them to the CTAs (CTA pairs
+// when PAIR) in forward order for even k and in reverse order for odd k (a
+// snake), so the one that got the longest item of a round gets the shortest of
+// the next.
+template <bool PAIR>
 __device__ __forceinline__ long long snake_item(long long rnd) {
-  const long long G = gridDim.x;
-  return rnd * G + ((rnd & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
+  const long long G = gridDim.x >> (PAIR ? 1 : 0);
+  const long long me = blockIdx.x >> (PAIR ? 1 : 0);
+  return rnd * G + ((rnd & 1) ? (G - 1 - me) : me);
 }
 
 struct Item {
@@ -215,16 +227,24 @@ struct Item {
   int t0, t1;       // this item's tile range
 };
 
-template <bool PAGED, bool CAND>
-__device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem) {
+// Item m of user b covers query rows [bm m, bm m + bm) with bm = BM, or, for a
+// CTA pair, bm = 2 BM rows of which CTA `rank` owns [bm m + BM rank, + BM).
+// Both CTAs of a pair derive the same key-tile range (that of the whole block);
+// rows of the lower half simply see more fully masked tiles.
+template <bool PAGED, bool CAND, bool PAIR>
+__device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem,
+                                          uint32_t rank) {
   Item it;
   it.b = b;
   it.m = m;
   it.h = rem / P.n_split;
   it.s = rem % P.n_split;
+  const int64_t bm = PAIR ? 2 * BM : BM;
   const int64_t qs = sm.m_q[b], nq = (int64_t)sm.m_q[b + 1] - qs;
-  it.q_row0 = qs + (int64_t)BM * m;
-  it.nvalid = (int)min64(BM, nq - (int64_t)BM * m);
+  const int64_t blk0 = bm * m;                           // first row of the block
+  const int64_t r0 = blk0 + (PAIR ? (int64_t)BM * rank : 0);  // first row of this CTA
+  it.q_row0 = qs + r0;
+  it.nvalid = (int)max64(0, min64(BM, nq - r0));
   it.n_k = sm.m_nk[b];
   if (PAGED) {
     it.user = sm.m_kv[b];
@@ -239,8 +259,9 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
     it.n_main = (int)((it.n_k + BN - 1) / BN);
     total = it.n_main + 1;
   } else {
-    it.p0 = it.n_k - nq + (int64_t)BM * m;
-    const int64_t last = it.p0 + it.nvalid - 1;
+    it.p0 = it.n_k - nq + r0;
+    // position of the block's last valid row
+    const int64_t last = it.n_k - nq + blk0 + min64(bm, nq - blk0) - 1;
     it.n_main = last >= 0 ? (int)(last / BN) + 1 : 0;
     total = it.n_main;
   }
@@ -252,6 +273,28 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
     it.t1 = total;
   }
   return it;
+}
+
+// MMA completion: one CTA's barrier, or the same barrier in both CTAs of a pair.
+template <bool PAIR>
+__device__ __forceinline__ void commit(uint32_t bar) {
+  if (PAIR)
+    umma_commit_pair(bar);
+  else
+    umma_commit(bar);
+}
+// Arrive on a barrier that CTA 0 of a pair owns (this CTA's own otherwise).
+template <bool PAIR>
+__device__ __forceinline__ void arrive_shared(uint32_t bar) {
+  if (PAIR)
+    mbar_arrive_cluster(mapa_shared(bar, 0));
+  else
+    mbar_arrive(bar);
+}
+// Wait on a barrier that both CTAs of a pair arrive on.
+template <bool PAIR>
+__device__ __forceinline__ bool wait_shared(uint32_t bar, uint32_t parity) {
+  return PAIR ? mbar_wait_cluster(bar, parity) : mbar_wait(bar, parity);
 }
 
 __device__ __forceinline__ void record_timeout(const KParams& P, Smem& sm) {
@@ -364,7 +407,7 @@ __device__ __forceinline__ void pw_chunk_any(const uint32_t (&sv)[16], uint32_t 
 }
 
 // ------------------------------------------------------------ the kernel
-template <bool PAGED, bool CAND>
+template <bool PAGED, bool CAND, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     hstu_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -374,8 +417,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
+  static_assert(!(PAIR && CAND), "CTA pairs serve the causal path only");
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  // rank in the CTA pair (0 issues the pair's MMAs and owns the shared barriers)
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
   // ---- setup
   for (int b = tid; b <= P.B; b += kThreads) {
@@ -410,17 +456,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.v_full[i]), 1);
       mbar_init(smem_u32(&sm.v_empty[i]), 1);
     }
-    for (int i = 0; i < 2 * NSP; ++i) mbar_init(smem_u32(&sm.s_full[i]), 1);
+    // P written / O drained: the 16 pointwise warps, of each CTA of a pair
     for (int i = 0; i < NSP; ++i) {
-      mbar_init(smem_u32(&sm.p_full[i]), 8);
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.p_full[i]), PAIR ? 32 : 16);
       mbar_init(smem_u32(&sm.sp_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.o_full[0]), 1);
-    mbar_init(smem_u32(&sm.o_full[1]), 1);
-    mbar_init(smem_u32(&sm.o_empty), 8);
+    mbar_init(smem_u32(&sm.o_full), 1);
+    mbar_init(smem_u32(&sm.o_empty), PAIR ? 32 : 16);
     for (int i = 0; i < NTS; ++i) {
       mbar_init(smem_u32(&sm.ts_full[i]), 1);
-      mbar_init(smem_u32(&sm.ts_empty[i]), 8);
+      mbar_init(smem_u32(&sm.ts_empty[i]), 16);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.qts_full[i]), 1);
@@ -438,35 +484,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&sm.tmem_base), 512);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(&sm.tmem_base), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&sm.tmem_base), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // the peer CTA signals barriers of CTA 0 only after both have initialised them
+  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int HS = P.H * P.n_split;
 
   if (warp == 0) {
     // =============================================== TMA producer
-    Sched sc;
+    Sched<PAIR ? 2 * BM : BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
-      const long long t = snake_item(rnd);
+      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
         const uint32_t qs = qi % QST;
         ok = mbar_wait(smem_u32(&sm.q_empty[qs]), ((qi / QST) & 1) ^ 1);
         if (ok) {
           const uint32_t bar = smem_u32(&sm.q_full[qs]);
-          mbar_arrive_expect_tx(bar, kTileBytes);
-          tma_load_3d(smem_u32(sm.q[qs]), &tm_q, bar, 0, it.h, (int)it.q_row0);
-          tma_load_3d(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
+          if (PAIR) {
+            // each CTA loads its own 128 rows; CTA 0's barrier counts both
+            const uint32_t lbar = mapa_shared(bar, 0);
+            if (rank == 0) mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+            tma_load_3d_pair(smem_u32(sm.q[qs]), &tm_q, lbar, 0, it.h, (int)it.q_row0);
+            tma_load_3d_pair(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, lbar, 64, it.h,
+                             (int)it.q_row0);
+          } else {
+            mbar_arrive_expect_tx(bar, kTileBytes);
+            tma_load_3d(smem_u32(sm.q[qs]), &tm_q, bar, 0, it.h, (int)it.q_row0);
+            tma_load_3d(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -503,13 +565,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = smem_u32(which == 0 ? sm.k[slot] : sm.v[slot]);
           if (lane == 0) {
             ok = mbar_wait(smem_u32(which == 0 ? &sm.k_empty[slot] : &sm.v_empty[slot]), par);
-            if (ok) mbar_arrive_expect_tx(bar, kTileBytes);
+            // a pair's tile is two 16 KiB halves, one per CTA, counted by CTA 0
+            if (ok && (!PAIR || rank == 0)) mbar_arrive_expect_tx(bar, kTileBytes);
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           if (which == 0) ++kc; else ++vc;
           const int half = lane & 1;
-          if (CAND && tile == it.n_main) {
+          if (PAIR) {
+            // K: keys [64 rank, 64 rank + 64) of the tile (pages 2 rank, 2 rank + 1),
+            //    both 64-column halves, as a 64-row K-major block per half;
+            // V: all four pages, value columns [64 rank, 64 rank + 64).
+            if (lane < 4) {
+              const int pg = which == 0 ? 2 * (int)rank + (lane >> 1) : lane;
+              const int idx = tile * 4 + pg;
+              const int si = (tile - it.t0) * 4 + pg;
+              const int32_t* plist = P.page_lists + it.user * (int64_t)P.max_ppu;
+              int64_t page = si < kPagesStaged ? (int64_t)sm.pages[si]
+                                               : (idx < P.max_ppu ? (int64_t)plist[idx] : -1);
+              if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
+              const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
+              const uint32_t lbar = mapa_shared(bar, 0);
+              if (which == 0)
+                tma_load_2d_pair(dst + half * kPairHalfK + (lane >> 1) * 4096, &tm_k, lbar,
+                                 half * 64, row);
+              else
+                tma_load_2d_pair(dst + lane * 4096, &tm_k, lbar, 64 * (int)rank, row);
+            }
+          } else if (CAND && tile == it.n_main) {
             if (lane < 2)
               tma_load_3d(dst + half * kHalfBytes, which == 0 ? &tm_kc : &tm_vc, bar, half * 64,
                           it.h, (int)it.q_row0);
@@ -534,7 +617,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-    if (!ok && lane == 0) {
+    if (!ok && lane == 0 && PAIR && rank != 0) {
+      // this CTA's copies signal CTA 0's barriers, which it cannot wait on:
+      // give any copy still in flight time to land before the CTA can exit
+      record_timeout(P, sm);
+      const unsigned long long t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
+      }
+    } else if (!ok && lane == 0) {
       record_timeout(P, sm);
       // let copies already in flight land before the CTA can exit
       for (uint32_t i = 0; i < KST && i < kc; ++i) {
@@ -554,16 +644,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =============================================== MMA issuers
     // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
     // tensor pipe fed: while one waits on its barriers the other's MMAs run.
-    Sched sc;
+    Sched<PAIR ? 2 * BM : BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
-    for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item(rnd);
+    // in a CTA pair only CTA 0 issues (M = 256 MMAs over both CTAs' operands)
+    for (long long rnd = 0; ok && (!PAIR || rank == 0); ++rnd) {
+      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
       if (it.t0 >= it.t1) continue;
       const int nt = it.t1 - it.t0;
       if (lane == 0) {
@@ -584,20 +675,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < HD / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
               const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-              const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-              umma_ss(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+              if (PAIR) {
+                // each CTA holds 64 keys: 64-row blocks per 64-column half
+                const uint32_t koff = (kk >> 2) * kPairHalfK + (kk & 3) * 32;
+                const uint64_t bdesc = smem_desc_sw128(k_base + koff, 16, 1024);
+                umma_ss_pair(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK2, kk > 0 ? 1u : 0u);
+              } else {
+                const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+                umma_ss(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+              }
             }
-            umma_commit(smem_u32(&sm.k_empty[slot]));
-            umma_commit(smem_u32(&sm.s_full[g % (2 * NSP)]));
-            if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
+            commit<PAIR>(smem_u32(&sm.k_empty[slot]));
+            commit<PAIR>(smem_u32(&sm.s_full[sb]));
+            if (i == nt - 1) commit<PAIR>(smem_u32(&sm.q_empty[qs]));
           }
         } else {
           for (int i = 0; i < nt && ok; ++i, ++g, ++vc) {
             const uint32_t pb = g % NSP;
             const uint32_t slot = vc % VST;
-            ok = mbar_wait(smem_u32(&sm.p_full[pb]), (g / NSP) & 1) &&
+            // P and drained-O arrivals come from both CTAs of a pair
+            ok = wait_shared<PAIR>(smem_u32(&sm.p_full[pb]), (g / NSP) & 1) &&
                  mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1) &&
-                 (i != 0 || mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
+                 (i != 0 || wait_shared<PAIR>(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
             if (!ok) break;
             tc_fence_after();
             const uint32_t v_base = smem_u32(sm.v[slot]);
@@ -605,26 +704,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BN / 16; ++kk) {
               // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key
               // groups 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
+              // (a CTA of a pair holds one 64-column half: the same layout)
               const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
-              umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV,
-                      (i == 0 && kk == 0) ? 0u : 1u);
+              if (PAIR)
+                umma_ts_pair(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV2,
+                             (i == 0 && kk == 0) ? 0u : 1u);
+              else
+                umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV,
+                        (i == 0 && kk == 0) ? 0u : 1u);
             }
-            umma_commit(smem_u32(&sm.v_empty[slot]));
-            umma_commit(smem_u32(&sm.sp_empty[pb]));
+            commit<PAIR>(smem_u32(&sm.v_empty[slot]));
+            commit<PAIR>(smem_u32(&sm.sp_empty[pb]));
           }
-          // the pair that processed the item's last key tile runs its epilogue
-          if (ok) umma_commit(smem_u32(&sm.o_full[(g - 1) & 1]));
+          if (ok) commit<PAIR>(smem_u32(&sm.o_full));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       g = __shfl_sync(0xffffffffu, g, 0);
       ++qi;
     }
-    if (lane == 0) {
+    if (lane == 0 && (!PAIR || rank == 0)) {
       if (!ok) record_timeout(P, sm);
       // all MMAs issued by this thread must finish before TMEM is released
       const uint32_t done = smem_u32(qk_role ? &sm.mma_done : &sm.mma_done2);
-      umma_commit(done);
+      commit<PAIR>(done);
       mbar_wait(done, 0);
     }
     __syncwarp();
@@ -633,15 +736,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Stages the key timestamps of every tile (in the MMA's tile order) for the
     // time-gap bias, so the pointwise warps never wait on global loads.
     if (P.time_table != nullptr && !PAGED && !CAND) {
-      Sched sc;
+      Sched<PAIR ? 2 * BM : BM> sc;
       sc.init(sm.m_q, P.B, HS, lane);
       uint32_t g = 0, qitem = 0;
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item(rnd);
+      const long long t = snake_item<PAIR>(rnd);
         int b, m, rem;
         if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-        const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+        const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
         if (it.t0 >= it.t1) continue;
         const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
         {  // query timestamps of this item's rows
@@ -711,32 +814,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // =============================================== pointwise + epilogue
-    // 16 warps: key tiles alternate between two pairs of warpgroups; within a
-    // pair, warpgroup `chalf` takes score columns [64 chalf, 64 chalf + 64).
+    // 16 warps share every key tile: warp (cq, sub) takes score columns
+    // [32 cq, 32 cq + 32) of tile rows [32 sub, 32 sub + 32), so each tile's
+    // SiLU finishes in the shortest time and the three S/P buffers let the
+    // tensor pipe run ahead.
     const int pwi = warp - 4;                       // 0..15
-    const int wg = pwi >> 3;                        // tile parity handled
-    const int chalf = (pwi >> 2) & 1;               // column half of the tile
+    const int cq = pwi >> 2;                        // column quarter of the tile
     const int sub = warp & 3;                       // TMEM lane quarter
     const int r = sub * 32 + lane;                  // tile row owned by this thread
+    const int cbase = 32 * cq;                      // first score column of this warp
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
     const bool use_pos = P.pos_table != nullptr;
     float* rrow = sm.rrow[pwi];
     const float self_rab = sm.pos_ext[0];
+    // offset that puts this warp's position-bias row at rrow[0 .. 63)
+    const int roff = 96 - cbase;
     // last position bucket this thread read, and its bias (tiles far from the
     // diagonal keep the same bucket for long runs, so the shared table is
     // rarely touched on the constant-row path)
     int pb_idx = -1;
     float pb_val = 0.f;
-    Sched sc;
+    Sched<PAIR ? 2 * BM : BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
-    uint32_t qi = 0, g = 0, my_epi = 0;
+    uint32_t qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item(rnd);
+      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
       if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
@@ -752,7 +859,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tq_exact = sm.qts[qsl].exact != 0;
       }
       for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
-        if ((int)(g & 1) != wg) continue;
         const uint32_t sb = g % NSP;
         const bool cand_tile = CAND && tile == it.n_main;
         const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
@@ -762,9 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t qp0 = CAND ? it.p0 : it.p0 + sub * 32;
         const int qrel0 = (int)max64(min64(qp0 - k0, 1 << 30), -(1 << 30));
         const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
-        // offset of this warp's column half in its position-bias row
-        const int roff = chalf ? 0 : 64;
-        // element (row lane, column c) reads rbase[127 - c]
+        // element (row lane, column c) reads rtab[rshift + 127 - c]
         const int rshift = use_pos ? ((CAND ? 0 : lane) - roff) : 0;
         const float* rtab = use_pos ? rrow : sm.pos_ext;  // zeros without a table
         const uint32_t tslot = g % NTS;
@@ -774,16 +878,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           time_fast = tq_exact && sm.ts[tslot].exact;
         }
-        // Far from the diagonal a row's 64 columns usually share one position
+        // Far from the diagonal a row's 32 columns usually share one position
         // bucket (and, with sorted key timestamps, one time bucket): then the
         // whole bias is one constant per row and is folded into the SiLU.
         float crow = 0.f;
         bool rowconst = false;
         if (!cand_tile) {
-          const int cbase = 64 * chalf;
-          const int dmax = qrel - cbase, dmin = qrel - cbase - 63;
+          const int dmax = qrel - cbase, dmin = qrel - cbase - 31;
           bool ok_row = dmin >= 0 || CAND;  // every column of both chunks visible
-          if (CAND) ok_row = cbase + 63 < kend;
+          if (CAND) ok_row = cbase + 31 < kend;
           if (use_pos) {
             const int b_hi = min(31 - __clz(max(dmax, 0) + 1), kMaxRab - 1);
             const int b_lo = min(31 - __clz(max(dmin, 0) + 1), kMaxRab - 1);
@@ -796,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (use_time) {
             const TsSlot& ts = sm.ts[tslot];
-            long long d_hi = tq_i - ts.i[cbase], d_lo = tq_i - ts.i[cbase + 63];
+            long long d_hi = tq_i - ts.i[cbase], d_lo = tq_i - ts.i[cbase + 31];
             d_hi = d_hi < 0 ? 0 : d_hi;
             d_lo = d_lo < 0 ? 0 : d_lo;
             const int t_hi = min(63 - __clzll(d_hi + 1), kMaxRab - 1);
@@ -807,8 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rowconst = __all_sync(0xffffffffu, ok_row);
         }
         // position-bias row of this warp, only needed off the constant-row path:
-        // rrow[j] = position bias at delta qrel0 + j + roff - 127; this warp's
-        // columns need j in [0, 95)
+        // rrow[j] = position bias at delta qrel0 + j + roff - 127, j in [0, 63)
         if (use_pos && !cand_tile && !rowconst) {
           __syncwarp();
 #pragma unroll
@@ -819,106 +921,76 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
         }
-        ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
+        // every pointwise warp waits every phase of s_full in order
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[sb]), (g / NSP) & 1);
         if (!ok) break;
         tc_fence_after();
-        // this warp's 64 S columns and, over their first half, its 32 P columns
-        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
+        // this warp's 32 S columns; its 16 P columns overwrite the first half
+        // (chunk q of P goes to columns [8q, 8q + 8), already loaded as S)
+        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + cbase;
         const uint32_t p_addr = s_addr;
         const float hrow = 0.5f * crow;
-        // Two 16-column chunks per (rolled) iteration: chunk q + 1 loads while
-        // chunk q computes.  P of chunk q goes to columns [8q, 8q + 8), which
-        // only covers S chunks already loaded into registers.
         uint32_t sa[16], sb2[16], pk[8];
         tmem_ld16(s_addr, sa);
+        tmem_ld16(s_addr + 16, sb2);
+        tmem_wait_ld();
+        reg_fence(sa);
+        reg_fence(sb2);
         if (rowconst) {
-#pragma unroll 1
-          for (int q = 0; q < 4; q += 2) {
-            tmem_wait_ld();
-            reg_fence(sa);
-            tmem_ld16(s_addr + (q + 1) * 16, sb2);
-            silu_rowconst(sa, pk, hrow);
-            tmem_st8(p_addr + q * 8, pk);
-            tmem_wait_ld();
-            reg_fence(sb2);
-            if (q == 0) tmem_ld16(s_addr + 32, sa);
-            silu_rowconst(sb2, pk, hrow);
-            tmem_st8(p_addr + (q + 1) * 8, pk);
-          }
+          silu_rowconst(sa, pk, hrow);
+          tmem_st8(p_addr, pk);
+          silu_rowconst(sb2, pk, hrow);
+          tmem_st8(p_addr + 8, pk);
         } else {
-          const int cb0 = chalf * 64;
-          const float* rl0 = rtab + (rshift + 127 - cb0);
+          const float* rl0 = rtab + (rshift + 127 - cbase);
           const TsSlot& ts = sm.ts[use_time ? tslot : 0];
           const int tmode = use_time ? (time_fast ? 1 : 2) : 0;
-#pragma unroll 1
-          for (int q = 0; q < 4; q += 2) {
-            tmem_wait_ld();
-            reg_fence(sa);
-            tmem_ld16(s_addr + (q + 1) * 16, sb2);
-            pw_chunk_any<CAND>(sa, pk, cb0 + q * 16, cand_tile, sub, qrel0, kend, tmode, rl0 - q * 16,
-                               qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
-            tmem_st8(p_addr + q * 8, pk);
-            tmem_wait_ld();
-            reg_fence(sb2);
-            if (q == 0) tmem_ld16(s_addr + 32, sa);
-            pw_chunk_any<CAND>(sb2, pk, cb0 + q * 16 + 16, cand_tile, sub, qrel0, kend, tmode,
-                               rl0 - q * 16 - 16, qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
-            tmem_st8(p_addr + (q + 1) * 8, pk);
-          }
+          pw_chunk_any<CAND>(sa, pk, cbase, cand_tile, sub, qrel0, kend, tmode, rl0, qrel, r, ts,
+                             tq1, tq_i, sm.time_ext, self_rab);
+          tmem_st8(p_addr, pk);
+          pw_chunk_any<CAND>(sb2, pk, cbase + 16, cand_tile, sub, qrel0, kend, tmode, rl0 - 16,
+                             qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
+          tmem_st8(p_addr + 8, pk);
         }
         if (use_time) {
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
         }
-        if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
+        if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.p_full[sb]));
       }
       if (!ok) break;
       if (use_time) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.qts_empty[qsl]));
       }
-      // ---- epilogue, by the pair that processed the item's last key tile (so
-      // the other pair can start the next item at once); this warp stores O
-      // columns [64 chalf, 64 chalf + 64) of its 32 rows.
-      if ((int)((g - 1) & 1) != wg) {
-        ++qi;
-        continue;
-      }
-      // each pair has its own o_full barrier and waits every one of its phases
-      // in order (a parity wait must never run two phases ahead or behind)
-      ok = mbar_wait_warp(smem_u32(&sm.o_full[wg]), my_epi & 1);
-      ++my_epi;
+      // ---- epilogue: this warp stores O columns [32 cq, 32 cq + 32) of its
+      // 32 rows (every warp waits every phase of o_full in order)
+      ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
       if (!ok) break;
       tc_fence_after();
       const bool row_ok = r < it.nvalid && it.q_row0 + r < P.total_q;
       const int64_t row = it.q_row0 + r;
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
-        const int ocol = 64 * chalf + 32 * q;
-        uint32_t oa[32];
-        tmem_ld32(tmem + lane_addr + TM_O + ocol, oa);
-        tmem_wait_ld();
-        reg_fence(oa);
-        if (q == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
-        }
-        if (!row_ok) continue;
+      uint32_t oa[32];
+      tmem_ld32(tmem + lane_addr + TM_O + cbase, oa);
+      tmem_wait_ld();
+      reg_fence(oa);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.o_empty));
+      if (row_ok) {
         if (P.partial) {
           float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
-                       it.h * HD + ocol;
+                       it.h * HD + cbase;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             reinterpret_cast<float4*>(dst)[j / 4] =
                 make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
                             __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
         } else {
-          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + ocol;
+          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + cbase;
           const float sc2 = P.scale;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
@@ -939,9 +1011,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  // a pair's MMAs write both CTAs' tensor memory and each CTA signals the
+  // other's barriers: neither releases anything before both are done
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -988,8 +1066,9 @@ __global__ void split_reduce_kernel(KParams P, int B) {
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-template <bool PAGED, bool CAND>
-cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, int grid, cudaStream_t stream) {
+template <bool PAGED, bool CAND, bool PAIR>
+cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items, int num_sms,
+                        cudaStream_t stream) {
   CUtensorMap tq, tk, tv, tkc, tvc;
   const uint64_t qrows = (uint64_t)std::max<int64_t>(p.total_q, 1);
   if (!make_tmap_3d(&tq, p.q, HD, p.H, qrows, HD * 2, (uint64_t)p.q_stride * 2, 64, BM))
@@ -1014,21 +1093,63 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, int grid, cudaS
     tkc = tq;
     tvc = tq;
   }
-  auto kern = hstu_attn_sm100_kernel<PAGED, CAND>;
+  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PAIR>;
   static bool attr_set[64] = {};
+  static int max_pairs[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  const bool cached = dev >= 0 && dev < 64 && attr_set[dev];
+  if (!cached) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes());
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<grid, kThreads, smem_bytes(), stream>>>(tq, tk, tv, tkc, tvc, kp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (!PAIR) {
+    const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
+    if (!cached && dev >= 0 && dev < 64) attr_set[dev] = true;
+    kern<<<grid, kThreads, smem_bytes(), stream>>>(tq, tk, tv, tkc, tvc, kp);
+    e = cudaGetLastError();
+  } else {
+    // persistent CTA pairs: as many 2-CTA clusters as can be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes();
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int pairs = cached ? max_pairs[dev] : 0;
+    if (!cached) {
+      cfg.gridDim = dim3(2 * (unsigned)std::max(1, num_sms / 2));
+      if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs <= 0) {
+        cudaGetLastError();
+        pairs = std::max(1, num_sms / 2);
+      }
+      if (dev >= 0 && dev < 64) {
+        max_pairs[dev] = pairs;
+        attr_set[dev] = true;
+      }
+    }
+    const long long n = std::max<long long>(1, std::min<long long>(items, pairs));
+    cfg.gridDim = dim3(2 * (unsigned)n);
+    e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tkc, tvc, kp);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
   if (e != cudaSuccess || kp.partial == nullptr) return e;
   split_reduce_kernel<PAGED><<<(unsigned)p.total_q, 128, 0, stream>>>(kp, p.B);
   return cudaGetLastError();
+}
+
+// -1 when HSTU_ATTN_CTA_PAIRS is unset, else 0 / 1.
+int cta_pair_override() {
+  const char* e = std::getenv("HSTU_ATTN_CTA_PAIRS");
+  if (e == nullptr || *e == 0) return -1;
+  return std::atoi(e) != 0 ? 1 : 0;
 }
 
 // Key-split plan for the candidate path: one wave of (user, head, split)
@@ -1110,15 +1231,22 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
     if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
     kp.partial = reinterpret_cast<float*>(workspace);
   }
-  const int qt = (p.max_q + BM - 1) / BM;
+  // Paged causal attention over long query runs may go to CTA pairs: each pair
+  // shares every K/V tile (each CTA loads half), halving the tile traffic into
+  // shared memory per SM.  HSTU_ATTN_CTA_PAIRS=1 / 0 forces the choice.
+  const bool eligible = p.paged && p.mode != 1 && p.max_q >= 2 * BM;
+  const int forced = cta_pair_override();
+  const bool pair = eligible && (forced >= 0 ? forced == 1 : kCtaPairsByDefault);
+  const int bm = pair ? 2 * BM : BM;
+  const int qt = (p.max_q + bm - 1) / bm;
   const long long items = (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
-  const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
   if (p.paged) {
-    return p.mode == 1 ? launch_impl<true, true>(p, kp, grid, stream)
-                       : launch_impl<true, false>(p, kp, grid, stream);
+    if (p.mode == 1) return launch_impl<true, true, false>(p, kp, items, num_sms, stream);
+    return pair ? launch_impl<true, false, true>(p, kp, items, num_sms, stream)
+                : launch_impl<true, false, false>(p, kp, items, num_sms, stream);
   }
-  return p.mode == 1 ? launch_impl<false, true>(p, kp, grid, stream)
-                     : launch_impl<false, false>(p, kp, grid, stream);
+  return p.mode == 1 ? launch_impl<false, true, false>(p, kp, items, num_sms, stream)
+                     : launch_impl<false, false, false>(p, kp, items, num_sms, stream);
 }
 
 }  // namespace hstu

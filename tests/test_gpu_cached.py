@@ -10,6 +10,10 @@ from tests.gpu_common import assert_bf16_close, assert_f32_close, dev, sample_ro
 
 pytestmark = pytest.mark.gpu
 
+# Causal launches with 256+ query rows can run on single CTAs or on CTA pairs
+# (HSTU_ATTN_CTA_PAIRS forces the choice); the causal tests cover both.
+CTA_PAIRS = pytest.mark.parametrize("cta_pairs", ["0", "1"])
+
 
 def prefill(table, case, users_t):
     """Alloc + append the pre-filled history (untimed set-up of every cached workload)."""
@@ -132,8 +136,10 @@ def test_candidates_workload_full_size():
     table.close()
 
 
+@CTA_PAIRS
 @pytest.mark.parametrize("lengths", [[64, 300, 1000], [17, 64, 129]])
-def test_causal_suffix_small(lengths):
+def test_causal_suffix_small(lengths, cta_pairs, monkeypatch):
+    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
     case = workloads.long_history(lengths=lengths, pool_tokens=4096)
     table = make_table(case)
     users = dev(case.users)
@@ -159,8 +165,44 @@ def test_causal_suffix_decode_queries_only():
     table.close()
 
 
-def test_long_history_workload_full_size_sampled():
+@CTA_PAIRS
+@pytest.mark.parametrize("lengths", [[255, 256, 257, 384, 385, 1], [1000, 130, 640]])
+def test_causal_suffix_query_blocks(lengths, cta_pairs, monkeypatch):
+    """Runs of 256+ queries go to CTA pairs (256-row blocks, one 128-row half per
+    CTA): block boundaries, a half with no valid rows, a lone row."""
+    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
+    case = workloads.long_history(lengths=lengths, pool_tokens=8192)
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), f"query blocks {lengths}", ulp_aware=True)
+    table.close()
+
+
+@CTA_PAIRS
+def test_causal_suffix_long_runs_behind_history(cta_pairs, monkeypatch):
+    """Query suffixes of 256-700 rows after long cached histories (block rows start
+    past position 0)."""
+    import dataclasses
+    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
+    case = workloads.long_history(lengths=[2000, 300, 3000], pool_tokens=8192)
+    nq = np.array([300, 256, 700], dtype=np.int64)
+    qo = workloads.offsets_from_lengths(case.total_lengths)
+    q = np.concatenate([case.q[qo[b + 1] - nq[b]:qo[b + 1]] for b in range(case.B)])
+    case = dataclasses.replace(case, q=q, n_q=nq)
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), "long suffixes", ulp_aware=True)
+    table.close()
+
+
+@CTA_PAIRS
+def test_long_history_workload_full_size_sampled(cta_pairs, monkeypatch):
     """32 users, Zipf lengths in [64,16384], 2M-token pool; oracle on sampled rows."""
+    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
     case = workloads.long_history()
     table = make_table(case)
     users = dev(case.users)
