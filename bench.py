@@ -45,6 +45,34 @@ WORKLOAD = ("long_history (B=32, L=clip(zipf(1.2),64,16384), H=4, d=128, bf16, p
             "history U[1024,4096], +64 appended, 128 candidates/user)")
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "generative_recommender_sequence_b200", "csrc", f)
+                  for f in ("attn_sm100.cu", "attn.h", "sm100.cuh")]
+
+
+def kernel_source_digest() -> str:
+    """SHA-256 over the attention kernel's sources (what an ncu capture was taken of)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu record,
+    or None when the record is missing or was taken on other kernel sources."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256") != kernel_source_digest():
+            return None
+        return int(rec["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -333,7 +361,7 @@ def run_gpu(args):
             "cached_candidates_per_s": round(cand_per_s * world, 1),
             "roofline": {"bound": "tensor", "kernel": "hstu_attn_sm100_kernel<paged, causal> (long_history)",
                          "achieved": round(a_attn_tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
-                         "frac": round(a_attn_tflops / tf_peak, 4), "traffic": None,
+                         "frac": round(a_attn_tflops / tf_peak, 4), "traffic": recorded_traffic(),
                          "peak_source": f"{peak_src} bf16 dense (burst)"},
             "gpu_launches": args.steps * 9,
             "clocks": clocks,
@@ -432,14 +460,15 @@ def run_oracle_sample(c5, rows5, c3, rows3, threads, kv5=None, kv3=None):
 def cpu_baseline(args):
     import oracle
     threads = oracle.default_threads()
-    c5, rows5, f5, c3, rows3, f3 = cpu_sample_units(rows_per_user=300, cands_per_user=32)
+    # about 10-15 s of fp64 work on a 16-core host
+    c5, rows5, f5, c3, rows3, f3 = cpu_sample_units(rows_per_user=2500, cands_per_user=32)
     kv5, kv3 = _joined_kv(c5), _joined_kv(c3)
     t0 = time.perf_counter()
     run_oracle_sample(c5, rows5, c3, rows3, threads, kv5, kv3)
     dt = time.perf_counter() - t0
     return {"value": round((f5 + f3) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"fp64 C oracle on {len(rows5)} query rows of long_history (up to 300 per user) + "
+            "sample": f"fp64 C oracle on {len(rows5)} query rows of long_history (up to 2500 per user) + "
                       f"{len(rows3)} candidates of cached_cand (32 per user); {dt:.1f} s"}
 
 
