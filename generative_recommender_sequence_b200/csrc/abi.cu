@@ -5,7 +5,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -23,7 +22,6 @@ struct hstu_kv_table {
   hstu::KvTableDev dev;
   int device;
   hstu_dtype dtype;
-  std::atomic<int32_t> epoch{1};
 };
 
 namespace hstu {
@@ -299,9 +297,8 @@ hstu_status hstu_kv_alloc(hstu_kv_table* t, const int64_t* users, const int64_t*
   if (B > 0 && (!users || !n_new_tokens)) return HSTU_ERR_INVALID_ARG;
   if (page_ids_out == nullptr) page_ids_cap = 0;
   if (B == 0 && page_ids_cap == 0) return HSTU_OK;
-  const int32_t epoch = t->epoch.fetch_add(1) + 1;
   return from_cuda(kv_alloc_launch(t->dev, users, n_new_tokens, B, page_ids_cap ? page_ids_out : nullptr,
-                                   page_ids_cap, epoch, stream));
+                                   page_ids_cap, stream));
 }
 
 hstu_status hstu_kv_append(hstu_kv_table* t, const int64_t* users, const void* k_new,

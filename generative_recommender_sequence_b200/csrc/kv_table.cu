@@ -13,6 +13,9 @@
 //   lengths     [max_users] int64 cached tokens
 //   epoch       [max_users] int32: last alloc call that listed the user
 //               (duplicate detection without clearing)
+//   alloc_calls int32 counter of alloc launches; each launch takes the next
+//               epoch from it on the device, so a captured and replayed
+//               launch still gets a fresh epoch
 //   done        [max_users] int32: append chunk counters (always back to 0)
 //   status      first device-side error since the last status read
 #include <cuda_bf16.h>
@@ -39,13 +42,18 @@ constexpr int kAllocThreads = 1024;
 // pages from the top of the free stack (user 0 first).
 __global__ void __launch_bounds__(kAllocThreads)
     kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new, int B,
-                    int32_t* page_ids_out, int page_ids_cap, int32_t epoch) {
+                    int32_t* page_ids_out, int page_ids_cap) {
   __shared__ int64_t s_chunk[kAllocThreads];
   __shared__ int s_bad;
+  __shared__ int s_epoch;
   __shared__ int64_t s_total;
   const int tid = threadIdx.x;
-  if (tid == 0) s_bad = 0;
+  if (tid == 0) {
+    s_bad = 0;
+    s_epoch = atomicAdd(t.alloc_calls, 1) + 1;
+  }
   __syncthreads();
+  const int32_t epoch = s_epoch;
   const int per = (B + kAllocThreads - 1) / kAllocThreads;
   const int b0 = tid * per, b1 = min(B, b0 + per);
   // phase 1
@@ -235,6 +243,10 @@ cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order
   if (e != cudaSuccess) return e;
   e = cudaMemset(t->epoch, 0, sizeof(int32_t) * (size_t)t->max_users);
   if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->alloc_calls, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->alloc_calls, 0, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
   e = cudaMalloc(&t->done, sizeof(int32_t) * (size_t)t->max_users);
   if (e != cudaSuccess) return e;
   e = cudaMemset(t->done, 0, sizeof(int32_t) * (size_t)t->max_users);
@@ -263,16 +275,15 @@ void kv_table_free_storage(KvTableDev* t) {
   cudaFree(t->n_held);
   cudaFree(t->lengths);
   cudaFree(t->epoch);
+  cudaFree(t->alloc_calls);
   cudaFree(t->done);
   cudaFree(t->status);
 }
 
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
-                            int32_t* page_ids_out, int page_ids_cap, int32_t epoch,
-                            cudaStream_t stream) {
+                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream) {
   if (B == 0 && page_ids_out == nullptr) return cudaSuccess;
-  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, B, page_ids_out, page_ids_cap,
-                                                   epoch);
+  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, B, page_ids_out, page_ids_cap);
   return cudaGetLastError();
 }
 

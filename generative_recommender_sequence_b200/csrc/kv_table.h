@@ -19,6 +19,7 @@ struct KvTableDev {
   int32_t* n_held;
   int64_t* lengths;
   int32_t* epoch;
+  int32_t* alloc_calls;  // device counter of alloc launches (the next call's epoch - 1)
   int32_t* done;
   int32_t* status;
 };
@@ -26,8 +27,7 @@ struct KvTableDev {
 cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order);
 void kv_table_free_storage(KvTableDev* t);
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
-                            int32_t* page_ids_out, int page_ids_cap, int32_t epoch,
-                            cudaStream_t stream);
+                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream);
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
                              const void* v_new, const int64_t* new_offsets, int B, int max_new,
                              cudaStream_t stream);

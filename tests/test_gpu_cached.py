@@ -236,3 +236,60 @@ def test_fp32_table_candidates_simt():
                                  pos_table=pt, scale=0.01)
     assert_f32_close(to_np(out), ref, "fp32 candidates")
     t.close()
+
+
+def test_step_replayed_from_a_cuda_graph():
+    """alloc + append + lookup + candidate attention captured once and replayed
+    twice: each replay appends the delta again into fresh pages (the alloc epoch
+    is taken on the device, so no replay looks like a duplicate user) and the
+    second replay scores the candidates over history + delta + delta."""
+    import dataclasses
+    import generative_recommender_sequence_b200 as hstu
+    base = workloads.cached_cand(B=3, hmin=0, hmax=1, n_new=40, n_cand=50, seed=11)
+    case = _with_lengths(base, np.array([100, 31, 300]), 40, 50, seed=12)
+    case = dataclasses.replace(case, n_pages=case.n_pages + 16,
+                               free_order=np.random.default_rng(13).permutation(case.n_pages + 16)
+                               .astype(np.int32))
+    mpp = int(np.max((case.total_lengths + case.n_new + 31) // 32)) + 2
+    table = hstu.KVTable(case.n_pages, case.H, case.d, max_users=case.B, max_pages_per_user=mpp,
+                         free_order=case.free_order)
+    users = dev(case.users)
+    prefill(table, case, users)
+    n_new, new_off = dev(case.n_new), dev(workloads.offsets_from_lengths(case.n_new))
+    new_k, new_v = storage(case.new_k, "bf16"), storage(case.new_v, "bf16")
+    q, kc, vc = (storage(x, "bf16") for x in (case.q_cand, case.k_cand, case.v_cand))
+    q_off, pt = dev(case.q_offsets), dev(case.pos_table)
+    max_cached = int((case.total_lengths + case.n_new).max())
+    lens = torch.empty(case.B, dtype=torch.int64, device="cuda")
+    ptab = torch.empty((case.B, mpp), dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    ws_bytes = table.workspace_size(case.B, int(case.q_offsets[-1]), int(case.n_cand.max()), max_cached,
+                                    hstu.HSTU_MASK_CANDIDATES)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+
+    def one_step():
+        table.alloc(users, n_new)
+        table.append(users, new_k, new_v, new_off, int(case.n_new.max()))
+        table.lookup(users, lens, ptab)
+        hstu.attn_cached_fwd(table, users, q, q_off, int(case.n_cand.max()), max_cached,
+                             hstu.HSTU_MASK_CANDIDATES, k_cand=kc, v_cand=vc, pos_table=pt,
+                             scale=case.scale, out=out, workspace=ws)
+
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        one_step()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert table.status() == 0
+    assert hstu.last_device_error() == 0
+    expect_len = case.hist_lengths + 2 * case.n_new
+    assert lens.cpu().numpy().tolist() == expect_len.tolist()
+    twice = dataclasses.replace(case, n_new=2 * case.n_new,
+                                new_k=np.concatenate([np.concatenate([case.new_k[40 * b:40 * b + 40]] * 2)
+                                                      for b in range(case.B)]),
+                                new_v=np.concatenate([np.concatenate([case.new_v[40 * b:40 * b + 40]] * 2)
+                                                      for b in range(case.B)]))
+    assert_bf16_close(to_np(out), oracle_out(twice), "graph replay", ulp_aware=True)
+    table.close()
