@@ -14,10 +14,11 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import (HSTU_BF16, HSTU_F32, HSTU_MASK_CANDIDATES, HSTU_MASK_CAUSAL_SUFFIX, HstuError,
-                   HstuRab, check, declared_symbols, load)
+from ._lib import (HSTU_BF16, HSTU_ERR_INVALID_ARG, HSTU_F32, HSTU_MASK_CANDIDATES,
+                   HSTU_MASK_CAUSAL_SUFFIX, HstuError, HstuRab, check, declared_symbols, load)
 
-__all__ = ["attn_fwd", "attn_cached_fwd", "KVTable", "block_fwd", "HstuError", "load",
+__all__ = ["attn_fwd", "attn_cached_fwd", "KVTable", "block_fwd", "block_cached_step",
+           "block_cached_workspace_size", "HstuError", "load",
            "declared_symbols", "device_check", "last_device_error",
            "HSTU_MASK_CANDIDATES", "HSTU_MASK_CAUSAL_SUFFIX"]
 
@@ -200,4 +201,58 @@ def block_fwd(x, seq_offsets, max_len: int, w_uvqk: Sequence[torch.Tensor],
                                float(scale), float(ln_eps), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream))
     check("hstu_block_fwd", st)
+    return x
+
+
+def _tables_array(tables: Sequence["KVTable"]):
+    arr = (ctypes.c_void_p * len(tables))(*[t.handle.value for t in tables])
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+def block_cached_workspace_size(tables: Sequence["KVTable"], B: int, T_new: int, T_cand: int,
+                                max_cand: int, max_cached: int, d_model: int = 512, H: int = 4,
+                                dh: int = 128) -> int:
+    arr, ptr = _tables_array(tables)
+    return load().hstu_block_cached_workspace_size(ptr, len(tables), B, T_new, T_cand, max_cand,
+                                                   max_cached, d_model, H, dh)
+
+
+def block_cached_step(tables: Sequence["KVTable"], users, x, new_offsets, max_new: int,
+                      cand_offsets, max_cand: int, max_cached: int, w_uvqk: Sequence[torch.Tensor],
+                      w_o: Sequence[torch.Tensor], pos_table=None, scale: float = 1.0,
+                      ln_eps: float = 1e-5, H: int = 4, dh: int = 128, T_new: Optional[int] = None,
+                      workspace=None, stream=None) -> torch.Tensor:
+    """KV-cached block step, in place on x = [new rows; candidate rows] (bf16).
+
+    tables[l] caches layer l's K/V; new_offsets / cand_offsets: [B+1] int64 device
+    (either may be None when there are no such rows).  T_new: number of new rows
+    (default: all rows when cand_offsets is None, else x rows minus candidates,
+    which needs cand_offsets on the host side as well - pass it explicitly)."""
+    _need_cuda(users, x, new_offsets, cand_offsets, *w_uvqk, *w_o)
+    T, dm = x.shape
+    L = len(w_uvqk)
+    if len(tables) != L or len(w_o) != L:
+        raise ValueError("one table, one w_uvqk and one w_o per layer")
+    if T_new is None:
+        if cand_offsets is not None:
+            raise ValueError("pass T_new when there are candidate rows")
+        T_new = T
+    T_cand = T - T_new
+    B = users.numel()
+    need = block_cached_workspace_size(tables, B, T_new, T_cand, max_cand, max_cached, dm, H, dh)
+    if need == 0:
+        raise HstuError("hstu_block_cached_workspace_size", HSTU_ERR_INVALID_ARG)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    arr, tptr = _tables_array(tables)
+    w1 = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_uvqk])
+    w2 = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_o])
+    rab = _rab(pos_table, None, None)
+    st = load().hstu_block_cached_step(
+        tptr, L, _ptr(users), B, _ptr(x), _ptr(new_offsets), int(T_new), int(max_new),
+        _ptr(cand_offsets), int(T_cand), int(max_cand), int(max_cached), dm, H, dh,
+        ctypes.cast(w1, ctypes.c_void_p), ctypes.cast(w2, ctypes.c_void_p),
+        ctypes.byref(rab) if rab else None, float(scale), float(ln_eps), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    check("hstu_block_cached_step", st)
     return x

@@ -61,6 +61,10 @@ _SIGNATURES = {
     "hstu_block_fwd": ([_P, _P, _I32, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _F, _F, _P,
                         _SZ, _P], _I32),
     "hstu_block_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
+    "hstu_block_cached_step": ([_P, _I32, _P, _I32, _P, _P, _I64, _I32, _P, _I64, _I32, _I32, _I32,
+                                _I32, _I32, _P, _P, _P, _F, _F, _P, _SZ, _P], _I32),
+    "hstu_block_cached_workspace_size": ([_P, _I32, _I32, _I64, _I64, _I32, _I32, _I32, _I32, _I32],
+                                         _SZ),
 }
 
 _lock = threading.Lock()

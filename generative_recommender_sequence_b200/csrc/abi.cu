@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "../../include/hstu.h"
 #include "attn.h"
@@ -442,6 +443,106 @@ hstu_status hstu_block_fwd(void* x, const int64_t* seq_offsets, int32_t B, int32
   p.scale = scale;
   p.ln_eps = ln_eps;
   const cudaError_t e = block_fwd_launch(p, workspace, ws_bytes, device_error_word(), stream);
+  if (e == cudaErrorNotSupported) return HSTU_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- cached multi-layer step
+namespace {
+
+// Host-side view of the per-layer tables; false if any table does not fit the block.
+bool cached_step_problem(hstu_kv_table* const* tables, int32_t n_layers, int32_t d_model, int32_t H,
+                         int32_t dh, std::vector<hstu::KvTableDev>* devs) {
+  if (!tables || n_layers <= 0) return false;
+  devs->clear();
+  for (int l = 0; l < n_layers; ++l) {
+    const hstu_kv_table* t = tables[l];
+    if (!t || t->dtype != HSTU_BF16 || t->dev.H != H || t->dev.d != dh || H * dh != d_model)
+      return false;
+    devs->push_back(t->dev);
+  }
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hstu_block_cached_workspace_size(hstu_kv_table* const* tables, int32_t n_layers, int32_t B,
+                                        int64_t T_new, int64_t T_cand, int32_t max_cand,
+                                        int32_t max_cached, int32_t d_model, int32_t H,
+                                        int32_t dh) {
+  std::vector<hstu::KvTableDev> devs;
+  if (B < 0 || T_new < 0 || T_cand < 0 || max_cand < 0 || max_cached < 0) return 0;
+  if (!cached_step_problem(tables, n_layers, d_model, H, dh, &devs)) return 0;
+  hstu::CachedStepProblem p;
+  p.tables = devs.data();
+  p.n_layers = n_layers;
+  p.B = B;
+  p.T_new = T_new;
+  p.T_cand = T_cand;
+  p.max_cand = max_cand;
+  p.max_cached = max_cached;
+  p.d_model = d_model;
+  p.H = H;
+  p.dh = dh;
+  return hstu::block_cached_workspace_bytes(p, hstu::device_sm_count());
+}
+
+hstu_status hstu_block_cached_step(hstu_kv_table* const* tables, int32_t n_layers,
+                                   const int64_t* users, int32_t B, void* x,
+                                   const int64_t* new_offsets, int64_t T_new, int32_t max_new,
+                                   const int64_t* cand_offsets, int64_t T_cand, int32_t max_cand,
+                                   int32_t max_cached, int32_t d_model, int32_t H, int32_t dh,
+                                   const void* const* w_uvqk, const void* const* w_o,
+                                   const hstu_rab* rab, float scale, float ln_eps, void* workspace,
+                                   size_t ws_bytes, cudaStream_t stream) {
+  if (n_layers < 0 || B < 0 || T_new < 0 || T_cand < 0 || max_new < 0 || max_cand < 0 ||
+      max_cached < 0 || d_model <= 0 || H <= 0 || dh <= 0)
+    return HSTU_ERR_INVALID_ARG;
+  if (T_new + T_cand >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
+  if (dh != 128 || H * dh != d_model || d_model != 512) return HSTU_ERR_UNSUPPORTED;
+  if (!rab_ok(rab, false)) return HSTU_ERR_UNSUPPORTED;
+  if (n_layers == 0 || B == 0 || T_new + T_cand == 0) return HSTU_OK;
+  if (B > hstu::kMaxCachedStepUsers) return HSTU_ERR_UNSUPPORTED;
+  std::vector<hstu::KvTableDev> devs;
+  if (!cached_step_problem(tables, n_layers, d_model, H, dh, &devs)) return HSTU_ERR_INVALID_ARG;
+  if (!users || !x || !aligned16(x) || !w_uvqk || !w_o) return HSTU_ERR_INVALID_ARG;
+  if ((T_new > 0 && (!new_offsets || max_new <= 0)) || (T_cand > 0 && (!cand_offsets || max_cand <= 0)))
+    return HSTU_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (!w_uvqk[l] || !w_o[l] || !aligned16(w_uvqk[l]) || !aligned16(w_o[l]))
+      return HSTU_ERR_INVALID_ARG;
+  hstu::CachedStepProblem p;
+  p.tables = devs.data();
+  p.n_layers = n_layers;
+  p.users = users;
+  p.B = B;
+  p.x = x;
+  p.new_offsets = new_offsets;
+  p.T_new = T_new;
+  p.max_new = max_new;
+  p.cand_offsets = cand_offsets;
+  p.T_cand = T_cand;
+  p.max_cand = max_cand;
+  p.max_cached = max_cached;
+  p.d_model = d_model;
+  p.H = H;
+  p.dh = dh;
+  p.w_uvqk = w_uvqk;
+  p.w_o = w_o;
+  if (rab && rab->pos_table) {
+    p.pos_table = rab->pos_table;
+    p.n_pos = rab->n_pos_buckets;
+  }
+  p.scale = scale;
+  p.ln_eps = ln_eps;
+  const size_t need = hstu::block_cached_workspace_bytes(p, hstu::device_sm_count());
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return HSTU_ERR_INVALID_ARG;
+  const cudaError_t e =
+      hstu::block_cached_step_launch(p, workspace, ws_bytes, device_error_word(), stream);
   if (e == cudaErrorNotSupported) return HSTU_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

@@ -359,4 +359,109 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
   return cudaSuccess;
 }
 
+namespace {
+
+// Paged attention over one layer's table for the rows described by (q, q_off).
+AttnProblem cached_attention(const CachedStepProblem& c, const KvTableDev& t, bool candidates,
+                             const __nv_bfloat16* rows, const int64_t* q_off, int64_t total_q,
+                             int max_q, __nv_bfloat16* out) {
+  const int F = c.H * c.dh;
+  AttnProblem a;
+  a.B = c.B;
+  a.H = c.H;
+  a.d = c.dh;
+  a.mode = candidates ? 1 : 0;
+  a.paged = true;
+  a.q_off = q_off;
+  a.users = c.users;
+  a.page_lists = t.page_lists;
+  a.lengths = t.lengths;
+  a.max_users = t.max_users;
+  a.max_ppu = t.max_ppu;
+  a.n_pages = t.n_pages;
+  a.pool = t.pool;
+  // rows hold [U | V | Q | K] blocks of F columns
+  a.q = rows + 2 * F;
+  a.k = candidates ? rows + 3 * F : nullptr;
+  a.v = candidates ? rows + F : nullptr;
+  a.q_stride = a.k_stride = a.v_stride = 4 * F;
+  a.total_q = total_q;
+  a.out = out;
+  a.out_stride = F;
+  a.pos_table = c.pos_table;
+  a.n_pos = c.n_pos;
+  a.scale = c.scale;
+  a.max_q = max_q;
+  a.max_kv = c.max_cached;
+  return a;
+}
+
+size_t block_part_bytes(int64_t T, int F) {
+  return align256((size_t)T * 4 * F * 2) + align256((size_t)T * F * 2) * 2;
+}
+
+}  // namespace
+
+size_t block_cached_workspace_bytes(const CachedStepProblem& p, int num_sms) {
+  const int F = p.H * p.dh;
+  size_t bytes = block_part_bytes(p.T_new + p.T_cand, F);
+  if (p.T_cand > 0 && p.n_layers > 0 && p.tables) {
+    const AttnProblem a = cached_attention(p, p.tables[0], true, nullptr, p.cand_offsets, p.T_cand,
+                                           p.max_cand, nullptr);
+    bytes += align256(attn_sm100_workspace_bytes(a, num_sms));
+  }
+  return bytes;
+}
+
+cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace, size_t ws_bytes,
+                                     int* err_word, cudaStream_t stream) {
+  const int F = p.H * p.dh;
+  if (p.dh != 128 || F != p.d_model || F != 512) return cudaErrorNotSupported;
+  const int64_t T = p.T_new + p.T_cand;
+  if (T == 0 || p.n_layers == 0) return cudaSuccess;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* uvqk = reinterpret_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)T * 4 * F * 2));
+  __nv_bfloat16* gate = reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)T * 4 * F * 2) +
+                                                         align256((size_t)T * F * 2));
+  uint8_t* split_ws = ws + block_part_bytes(T, F);
+  const size_t split_bytes = ws_bytes > block_part_bytes(T, F) ? ws_bytes - block_part_bytes(T, F) : 0;
+  __nv_bfloat16* cand_rows = uvqk + p.T_new * 4 * F;
+  const int M = (int)T;
+  for (int l = 0; l < p.n_layers; ++l) {
+    const KvTableDev& t = p.tables[l];
+    // [U | V | Q | K] = SiLU(X W1) for the new and the candidate rows at once
+    cudaError_t e = gemm_launch<EPI_SILU>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+                                          p.d_model, err_word, stream);
+    if (e != cudaSuccess) return e;
+    if (p.T_new > 0) {
+      // the new tokens' K, V join this layer's cache, then they attend causally
+      // over the cached history and themselves
+      e = kv_alloc_launch(t, p.users, nullptr, p.B, nullptr, 0, stream, p.new_offsets);
+      if (e != cudaSuccess) return e;
+      e = kv_append_launch(t, p.users, uvqk + 3 * F, uvqk + F, p.new_offsets, p.B, p.max_new, stream,
+                           4 * F);
+      if (e != cudaSuccess) return e;
+      const AttnProblem a =
+          cached_attention(p, t, false, uvqk, p.new_offsets, p.T_new, p.max_new, attn);
+      e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
+      if (e != cudaSuccess) return e;
+    }
+    if (p.T_cand > 0) {
+      // candidates see the cached history (new tokens included) and themselves
+      const AttnProblem a = cached_attention(p, t, true, cand_rows, p.cand_offsets, p.T_cand,
+                                             p.max_cand, attn + p.T_new * F);
+      e = attn_sm100_launch(a, split_ws, split_bytes, err_word, stream);
+      if (e != cudaSuccess) return e;
+    }
+    ln_gate_kernel<<<(unsigned)((T + 7) / 8), 256, 0, stream>>>(attn, uvqk, 4 * F, gate, T, p.ln_eps);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+                                  err_word, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace hstu

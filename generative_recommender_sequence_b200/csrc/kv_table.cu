@@ -41,8 +41,8 @@ constexpr int kAllocThreads = 1024;
 // exclusive scan of the demand in the order users are listed.  Phase 3: pop
 // pages from the top of the free stack (user 0 first).
 __global__ void __launch_bounds__(kAllocThreads)
-    kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new, int B,
-                    int32_t* page_ids_out, int page_ids_cap) {
+    kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new,
+                    const int64_t* new_offsets, int B, int32_t* page_ids_out, int page_ids_cap) {
   __shared__ int64_t s_chunk[kAllocThreads];
   __shared__ int s_bad;
   __shared__ int s_epoch;
@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(kAllocThreads)
   // phase 1
   int64_t mysum = 0;
   for (int b = b0; b < b1; ++b) {
-    const int64_t u = users[b], n = n_new[b];
+    const int64_t u = users[b];
+    const int64_t n = n_new ? n_new[b] : new_offsets[b + 1] - new_offsets[b];
     if (u < 0 || u >= t.max_users || n < 0) {
       atomicOr(&s_bad, 1);
       continue;
@@ -96,7 +97,8 @@ __global__ void __launch_bounds__(kAllocThreads)
   int64_t pre = s_chunk[tid] - mysum;  // exclusive prefix of this thread's first user
   for (int b = b0; b < b1; ++b) {
     const int64_t u = users[b];
-    const int64_t want = (t.lengths[u] + n_new[b] + t.page_size - 1) / t.page_size;
+    const int64_t n = n_new ? n_new[b] : new_offsets[b + 1] - new_offsets[b];
+    const int64_t want = (t.lengths[u] + n + t.page_size - 1) / t.page_size;
     int64_t need = want - t.n_held[u];
     need = need < 0 ? 0 : need;
     const int held = t.n_held[u];
@@ -122,7 +124,7 @@ constexpr int kCopyThreads = 256;
 template <int ESZ>
 __global__ void __launch_bounds__(kCopyThreads)
     kv_append_kernel(KvTableDev t, const int64_t* users, const uint8_t* k_new, const uint8_t* v_new,
-                     const int64_t* new_offsets) {
+                     const int64_t* new_offsets, int64_t src_row_bytes) {
   const int b = blockIdx.y;
   const int64_t u = users[b];
   const int64_t s = new_offsets[b], n = new_offsets[b + 1] - s;
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kCopyThreads)
       const int64_t pos = len + tok0 + tk;
       const int32_t page = t.page_lists[u * (int64_t)t.max_ppu + pos / t.page_size];
       const int slot = (int)(pos % t.page_size);
-      const uint8_t* src = (kv ? v_new : k_new) + src_row * (int64_t)t.H * t.d * ESZ;
+      const uint8_t* src = (kv ? v_new : k_new) + src_row * src_row_bytes;
       const uint4 x = reinterpret_cast<const uint4*>(src)[v];
       uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
                      ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
@@ -281,23 +283,30 @@ void kv_table_free_storage(KvTableDev* t) {
 }
 
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
-                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream) {
+                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream,
+                            const int64_t* new_offsets) {
   if (B == 0 && page_ids_out == nullptr) return cudaSuccess;
-  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, B, page_ids_out, page_ids_cap);
+  if (n_new == nullptr && new_offsets == nullptr) return cudaErrorInvalidValue;
+  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, new_offsets, B, page_ids_out,
+                                                   page_ids_cap);
   return cudaGetLastError();
 }
 
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
                              const void* v_new, const int64_t* new_offsets, int B, int max_new,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, int64_t src_row_elems) {
   if (B == 0 || max_new <= 0) return cudaSuccess;
+  const int64_t row_elems = src_row_elems > 0 ? src_row_elems : (int64_t)t.H * t.d;
+  // 16-byte vector copies: every source row must start on a 16-byte boundary
+  if (row_elems < (int64_t)t.H * t.d || (row_elems * t.esize) % 16 != 0)
+    return cudaErrorInvalidValue;
   dim3 grid((max_new + kAppendTok - 1) / kAppendTok, B);
   if (t.esize == 2)
     kv_append_kernel<2><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets);
+        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 2);
   else
     kv_append_kernel<4><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets);
+        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 4);
   return cudaGetLastError();
 }
 

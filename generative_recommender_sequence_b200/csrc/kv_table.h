@@ -26,11 +26,14 @@ struct KvTableDev {
 
 cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order);
 void kv_table_free_storage(KvTableDev* t);
+// n_new[b] tokens per user, or (n_new == nullptr) new_offsets[b + 1] - new_offsets[b].
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
-                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream);
+                            int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream,
+                            const int64_t* new_offsets = nullptr);
+// k_new / v_new rows are src_row_elems elements apart (0: H * d, packed rows).
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
                              const void* v_new, const int64_t* new_offsets, int B, int max_new,
-                             cudaStream_t stream);
+                             cudaStream_t stream, int64_t src_row_elems = 0);
 cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
                              int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
                              void* k_out, void* v_out, const int64_t* out_offsets, int max_len,

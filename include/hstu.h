@@ -242,6 +242,50 @@ HSTU_API hstu_status hstu_block_fwd(void* x, const int64_t* seq_offsets, int32_t
                            size_t ws_bytes, cudaStream_t stream);
 HSTU_API size_t hstu_block_workspace_size(int64_t T, int32_t d_model, int32_t H, int32_t dh);
 
+/*
+ * KV-cached serving step of the block stack ("NVIDIA Dynamo-Triton Gets
+ * End-to-End HSTU Generative Recommender Workflow", sections "What the workflow
+ * combines" and the benchmark: reusable key-value state is cached per layer so
+ * long histories are not recomputed when new tokens arrive).  For each layer l:
+ *   [U|V|Q|K] = SiLU(X @ w_uvqk[l]) for every row of x (new and candidate rows);
+ *   the new rows' K, V are allocated pages in tables[l] and appended after the
+ *     user's cached tokens;
+ *   new rows attend causally over the user's cached tokens and the new rows
+ *     (HSTU_MASK_CAUSAL_SUFFIX); candidate rows attend over the cached tokens
+ *     (new ones included) and themselves only (HSTU_MASK_CANDIDATES: every
+ *     candidate sits one position past the last cached token);
+ *   G = LayerNorm(A) * U;  X = X + G @ w_o[l].
+ * The result equals the uncached stack run over each user's whole sequence,
+ * each candidate appended last on its own.
+ *
+ * tables: HOST array of n_layers tables (bf16, H heads of dh, one per layer),
+ *   holding the same users with the same cached lengths.  A prefill is a call
+ *   with no candidates on empty tables, the history passed as the new rows.
+ * users: [B] device.  x: [T_new + T_cand, d_model] bf16, updated in place: the
+ *   new rows (jagged by new_offsets, [B+1] device) first, then the candidate
+ *   rows (jagged by cand_offsets, [B+1] device, counted from the first
+ *   candidate row).  max_new / max_cand: per-user bounds.  max_cached: bound on
+ *   any user's cached length after this step's append.
+ * rab: position table only (no time term).  scale = 1/N for the attention.
+ * Needs dh == 128, H*dh == d_model == 512, B <= 65535.
+ * workspace: >= hstu_block_cached_workspace_size(...) bytes (0 = invalid
+ *   arguments).  Page shortage or a duplicate user is recorded in the table's
+ *   status word (read it with hstu_kv_table_status per layer).
+ */
+HSTU_API hstu_status hstu_block_cached_step(hstu_kv_table* const* tables, int32_t n_layers,
+                                            const int64_t* users, int32_t B, void* x,
+                                            const int64_t* new_offsets, int64_t T_new,
+                                            int32_t max_new, const int64_t* cand_offsets,
+                                            int64_t T_cand, int32_t max_cand, int32_t max_cached,
+                                            int32_t d_model, int32_t H, int32_t dh,
+                                            const void* const* w_uvqk, const void* const* w_o,
+                                            const hstu_rab* rab, float scale, float ln_eps,
+                                            void* workspace, size_t ws_bytes, cudaStream_t stream);
+HSTU_API size_t hstu_block_cached_workspace_size(hstu_kv_table* const* tables, int32_t n_layers,
+                                                 int32_t B, int64_t T_new, int64_t T_cand,
+                                                 int32_t max_cand, int32_t max_cached,
+                                                 int32_t d_model, int32_t H, int32_t dh);
+
 #ifdef __cplusplus
 }
 #endif

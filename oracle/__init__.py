@@ -13,6 +13,8 @@ Contents
   per-user page lists, byte-exact pool).
 * ``brute.py``: an independent numpy restatement used only to cross-check the C
   code on tiny inputs.
+* ``cached.py``: the KV-cached multi-layer serving step, defined as the
+  uncached block stack over whole sequences (``hstu_block_cached``).
 
 Parity status: every function here is pinned by tests under
 ``tests/test_oracle_*.py`` (closed forms, reductions to library routines,
