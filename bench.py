@@ -268,6 +268,95 @@ class JaggedPart:
                            time_table=self.tt, timestamps=self.ts, scale=c.scale, out=self.out)
 
 
+class CachedServingPart:
+    """KV-cached multi-layer serving vs the same stack without the cache (the
+    pages' benchmark, on synthetic inputs): 8 users with histories U[1024, 8192]
+    cached per layer, each request adding 64 new tokens and scoring 128
+    candidates; hidden 512, 4 heads of 128, bf16.  The uncached path runs the
+    block over each user's whole sequence [history; new; candidates].  Both are
+    replayed from CUDA graphs; the prefill of the caches is not timed."""
+
+    def __init__(self, n_layers, n_runs, seed=2024):
+        import torch
+        import generative_recommender_sequence_b200 as hstu
+        import workloads as W
+        rng = np.random.default_rng(seed)
+        self.hstu, self.n_layers = hstu, n_layers
+        B, n_new, n_cand, dm = 8, 64, 128, 512
+        hist = rng.integers(1024, 8193, B).astype(np.int64)
+        bf = lambda a: W.to_torch(W._as_storage(np.asarray(a, np.float32), "bf16"), "bf16").cuda()
+        off = lambda n: torch.as_tensor(np.concatenate([[0], np.cumsum(n)]).astype(np.int64)).cuda()
+        x_hist = bf(rng.standard_normal((int(hist.sum()), dm)))
+        x_new = bf(rng.standard_normal((B * n_new, dm)))
+        x_cand = bf(rng.standard_normal((B * n_cand, dm)))
+        self.w1 = [bf(rng.normal(0, 0.02, (dm, 2048))) for _ in range(n_layers)]
+        self.w2 = [bf(rng.normal(0, 0.02, (512, dm))) for _ in range(n_layers)]
+        self.pt = torch.as_tensor(rng.normal(0, 0.1, 16).astype(np.float32)).cuda()
+        full_len = hist + n_new + n_cand
+        self.scale = 1.0 / int(full_len.max())
+        grow = n_new * (n_runs + 4)
+        self.max_cached = int(hist.max()) + grow
+        mpp = (self.max_cached + 31) // 32 + 2
+        n_pages = int(np.sum((hist + grow + 31) // 32)) + 8
+        self.tables = [hstu.KVTable(n_pages, 4, 128, max_users=B, max_pages_per_user=mpp)
+                       for _ in range(n_layers)]
+        self.users = torch.arange(B, dtype=torch.int64, device="cuda")
+        hstu.block_cached_step(self.tables, self.users, x_hist, off(hist), int(hist.max()), None, 0,
+                               int(hist.max()), self.w1, self.w2, pos_table=self.pt, scale=self.scale)
+        self.new_off, self.cand_off = off(np.full(B, n_new)), off(np.full(B, n_cand))
+        self.n_new, self.n_cand, self.T_new = n_new, n_cand, B * n_new
+        self.x0 = torch.cat([x_new, x_cand])
+        self.x = self.x0.clone()
+        self.ws = torch.empty(hstu.block_cached_workspace_size(self.tables, B, B * n_new, B * n_cand,
+                                                                n_cand, self.max_cached),
+                              dtype=torch.uint8, device="cuda")
+        # uncached: every user's whole sequence, candidates last
+        xh = x_hist.split(hist.tolist())
+        xn, xc = x_new.split(n_new), x_cand.split(n_cand)
+        self.full0 = torch.cat([torch.cat([xh[b], xn[b], xc[b]]) for b in range(B)])
+        self.full = self.full0.clone()
+        self.full_off, self.full_max = off(full_len), int(full_len.max())
+        self.ws_full = torch.empty(hstu.block_workspace_size(int(full_len.sum()), dm, 4, 128),
+                                   dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def cached(self):
+        self.hstu.block_cached_step(self.tables, self.users, self.x, self.new_off, self.n_new,
+                                    self.cand_off, self.n_cand, self.max_cached, self.w1, self.w2,
+                                    pos_table=self.pt, scale=self.scale, T_new=self.T_new,
+                                    workspace=self.ws)
+
+    def uncached(self):
+        self.hstu.block_fwd(self.full, self.full_off, self.full_max, self.w1, self.w2,
+                            pos_table=self.pt, scale=self.scale, workspace=self.ws_full)
+
+    def measure(self, runs):
+        import torch
+        self.cached()
+        self.uncached()
+        torch.cuda.synchronize()
+        g_c, g_u = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_c):
+            self.cached()
+        with torch.cuda.graph(g_u):
+            self.uncached()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        res = {}
+        for name, g, x, x0 in (("cached", g_c, self.x, self.x0), ("uncached", g_u, self.full, self.full0)):
+            tot = 0.0
+            for _ in range(runs):
+                x.copy_(x0)
+                e0.record(); g.replay(); e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1)
+            res[name + "_ms"] = round(tot / runs, 4)
+        for t in self.tables:
+            if t.status():
+                raise RuntimeError("KV table error in the cached serving measurement")
+        res["speedup"] = round(res["uncached_ms"] / res["cached_ms"], 2)
+        return res
+
+
 def run_gpu(args):
     import torch
     import workloads as W
@@ -353,6 +442,14 @@ def run_gpu(args):
         jt += e0.elapsed_time(e1) / 1e3
     jsteps = max(3, args.steps // 2)
 
+    # KV-cached multi-layer serving vs the uncached stack, reported beside the step
+    serving = {}
+    if not args.no_serving:
+        for n_layers in (3, 8):
+            part = CachedServingPart(n_layers, n_runs=5)
+            serving[f"layers_{n_layers}"] = part.measure(runs=5)
+            del part
+
     e2e = run_e2e(A, Bp, flush_buf, args) if rank == 0 else None
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
@@ -376,6 +473,7 @@ def run_gpu(args):
                 "cached_candidates": {"ms": round(t_b / args.steps * 1e3, 4),
                                       "candidates_per_s": round(cand_per_s, 1),
                                       "hbm_gbs": round(b_gbs, 1), "frac_of_hbm": round(b_gbs / hbm_peak, 4)},
+                "cached_serving": serving,
                 "jagged_bf16": {"ms": round(jt / jsteps * 1e3, 4),
                                 "tflops": round(J.flops * jsteps / jt / 1e12, 2),
                                 "frac_of_bf16_peak": round(J.flops * jsteps / jt / 1e12 / tf_peak, 4)},
@@ -531,6 +629,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
+    ap.add_argument("--no-serving", action="store_true",
+                    help="skip the cached vs uncached multi-layer serving report")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1044,7 +1044,16 @@ __global__ void split_reduce_kernel(KParams P, int B) {
   } else {
     n_k = P.kv_off[b + 1] - P.kv_off[b];
   }
-  const int total = (int)((n_k + BN - 1) / BN) + 1;  // candidate layout: history tiles + 1
+  int total;  // key tiles of this row's item, as make_item counts them
+  if (P.mode == 1) {
+    total = (int)((n_k + BN - 1) / BN) + 1;  // candidate layout: history tiles + 1
+  } else {
+    // causal suffix: the item's tiles run up to its query tile's last row
+    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
+    const int64_t m = (row - P.q_off[b]) / BM;
+    const int64_t last = n_k - nq + min64(BM * (m + 1), nq) - 1;
+    total = last >= 0 ? (int)(last / BN) + 1 : 0;
+  }
   const int n_valid = min(P.n_split, (total + P.kps - 1) / P.kps);
   const int F = P.H * HD;
   for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
@@ -1152,14 +1161,15 @@ int cta_pair_override() {
   return std::atoi(e) != 0 ? 1 : 0;
 }
 
-// Key-split plan for the candidate path: one wave of (user, head, split)
-// items, each streaming a long run of key tiles (fewer pipeline start-ups and
-// fewer partial sums than many short splits).
+// Key-split plan: one wave of (user, head, split) items, each streaming a long
+// run of key tiles (fewer pipeline start-ups and fewer partial sums than many
+// short splits).  Used by the candidate path and by causal runs of at most one
+// query tile per user (new tokens over a long cached history).
 void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
   *n_split = 1;
   *kps = 1 << 30;
-  if (p.mode != 1) return;
-  const int max_tiles = (p.max_kv + BN - 1) / BN + 1;
+  if (p.mode != 1 && p.max_q > BM) return;
+  const int max_tiles = (p.max_kv + BN - 1) / BN + (p.mode == 1 ? 1 : 0);
   const int qt = std::max(1, (p.max_q + BM - 1) / BM);
   const long long base_items = (long long)p.B * p.H * qt;
   if (base_items <= 0) return;

@@ -405,12 +405,21 @@ size_t block_part_bytes(int64_t T, int F) {
 size_t block_cached_workspace_bytes(const CachedStepProblem& p, int num_sms) {
   const int F = p.H * p.dh;
   size_t bytes = block_part_bytes(p.T_new + p.T_cand, F);
-  if (p.T_cand > 0 && p.n_layers > 0 && p.tables) {
-    const AttnProblem a = cached_attention(p, p.tables[0], true, nullptr, p.cand_offsets, p.T_cand,
-                                           p.max_cand, nullptr);
-    bytes += align256(attn_sm100_workspace_bytes(a, num_sms));
+  // key-split partials of either attention (they run one after the other)
+  size_t split = 0;
+  if (p.n_layers > 0 && p.tables) {
+    if (p.T_new > 0) {
+      const AttnProblem a = cached_attention(p, p.tables[0], false, nullptr, p.new_offsets, p.T_new,
+                                             p.max_new, nullptr);
+      split = std::max(split, attn_sm100_workspace_bytes(a, num_sms));
+    }
+    if (p.T_cand > 0) {
+      const AttnProblem a = cached_attention(p, p.tables[0], true, nullptr, p.cand_offsets,
+                                             p.T_cand, p.max_cand, nullptr);
+      split = std::max(split, attn_sm100_workspace_bytes(a, num_sms));
+    }
   }
-  return bytes;
+  return bytes + align256(split);
 }
 
 cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace, size_t ws_bytes,
@@ -444,7 +453,7 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
       if (e != cudaSuccess) return e;
       const AttnProblem a =
           cached_attention(p, t, false, uvqk, p.new_offsets, p.T_new, p.max_new, attn);
-      e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
+      e = attn_sm100_launch(a, split_ws, split_bytes, err_word, stream);
       if (e != cudaSuccess) return e;
     }
     if (p.T_cand > 0) {

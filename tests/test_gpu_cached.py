@@ -293,3 +293,20 @@ def test_step_replayed_from_a_cuda_graph():
                                                       for b in range(case.B)]))
     assert_bf16_close(to_np(out), oracle_out(twice), "graph replay", ulp_aware=True)
     table.close()
+
+
+def test_causal_suffix_short_runs_split_over_keys():
+    """At most one query tile per user: the keys are split over one wave of items
+    and the fp32 partials reduced per row (ragged runs, a user with no query)."""
+    import dataclasses
+    case = workloads.long_history(lengths=[3000, 40, 129, 700], pool_tokens=8192)
+    nq = np.array([128, 40, 1, 0], dtype=np.int64)
+    qo = workloads.offsets_from_lengths(case.total_lengths)
+    q = np.concatenate([case.q[qo[b + 1] - nq[b]:qo[b + 1]] for b in range(case.B)])
+    case = dataclasses.replace(case, q=q, n_q=nq)
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), "short causal runs", ulp_aware=True)
+    table.close()
