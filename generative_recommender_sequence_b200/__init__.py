@@ -141,6 +141,12 @@ class KVTable:
                                      _ptr(new_offsets), users.numel(), int(max_new), _stream(stream))
         check("hstu_kv_append", st)
 
+    def release(self, users, stream=None):
+        """Evict whole users: every page of each listed user returns to the free stack."""
+        _need_cuda(users)
+        check("hstu_kv_release", self.lib.hstu_kv_release(self.handle, _ptr(users), users.numel(),
+                                                          _stream(stream)))
+
     def lookup(self, users, cached_len_out=None, page_table_out=None, k_out=None, v_out=None,
                out_offsets=None, max_len: int = 0, stream=None):
         _need_cuda(users, cached_len_out, page_table_out, k_out, v_out, out_offsets)

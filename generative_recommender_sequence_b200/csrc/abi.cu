@@ -302,6 +302,14 @@ hstu_status hstu_kv_alloc(hstu_kv_table* t, const int64_t* users, const int64_t*
                                    page_ids_cap, stream));
 }
 
+hstu_status hstu_kv_release(hstu_kv_table* t, const int64_t* users, int32_t B,
+                            cudaStream_t stream) {
+  if (!t || B < 0 || B > 65536) return HSTU_ERR_INVALID_ARG;
+  if (B == 0) return HSTU_OK;
+  if (!users) return HSTU_ERR_INVALID_ARG;
+  return from_cuda(kv_release_launch(t->dev, users, B, stream));
+}
+
 hstu_status hstu_kv_append(hstu_kv_table* t, const int64_t* users, const void* k_new,
                            const void* v_new, const int64_t* new_offsets, int32_t B,
                            int32_t max_new, cudaStream_t stream) {

@@ -116,6 +116,69 @@ __global__ void __launch_bounds__(kAllocThreads)
   if (tid == 0) *t.free_top = (int32_t)(top - total);
 }
 
+// One CTA.  Releases every page of the listed users (eviction of whole users):
+// pages go back on the free stack in the order users are listed, each user's
+// pages from its last to its first, so its first page ends on top.  Lengths and
+// page lists are cleared.  Duplicate or out-of-range users leave the table
+// unchanged and set the status word.
+__global__ void __launch_bounds__(kAllocThreads)
+    kv_release_kernel(KvTableDev t, const int64_t* users, int B) {
+  __shared__ int64_t s_chunk[kAllocThreads];
+  __shared__ int s_bad;
+  __shared__ int s_epoch;
+  __shared__ int64_t s_total;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = 0;
+    s_epoch = atomicAdd(t.alloc_calls, 1) + 1;
+  }
+  __syncthreads();
+  const int32_t epoch = s_epoch;
+  const int per = (B + kAllocThreads - 1) / kAllocThreads;
+  const int b0 = tid * per, b1 = min(B, b0 + per);
+  int64_t mysum = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int64_t u = users[b];
+    if (u < 0 || u >= t.max_users) {
+      atomicOr(&s_bad, 1);
+      continue;
+    }
+    if (atomicExch(&t.epoch[u], epoch) == epoch) atomicOr(&s_bad, 1);  // listed twice
+    mysum += t.n_held[u];
+  }
+  s_chunk[tid] = mysum;
+  __syncthreads();
+  for (int off = 1; off < kAllocThreads; off <<= 1) {
+    const int64_t x = tid >= off ? s_chunk[tid - off] : 0;
+    __syncthreads();
+    s_chunk[tid] += x;
+    __syncthreads();
+  }
+  if (tid == kAllocThreads - 1) s_total = s_chunk[tid];
+  __syncthreads();
+  const int64_t total = s_total;
+  const int64_t top = *t.free_top;
+  if (s_bad || top + total > t.n_pages) {
+    if (tid == 0) set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
+    return;
+  }
+  int64_t pre = s_chunk[tid] - mysum;
+  for (int b = b0; b < b1; ++b) {
+    const int64_t u = users[b];
+    const int held = t.n_held[u];
+    int32_t* list = t.page_lists + u * (int64_t)t.max_ppu;
+    for (int k = 0; k < held; ++k) {
+      t.free_stack[top + pre + (held - 1 - k)] = list[k];
+      list[k] = -1;
+    }
+    t.n_held[u] = 0;
+    t.lengths[u] = 0;
+    pre += held;
+  }
+  __syncthreads();
+  if (tid == 0) *t.free_top = (int32_t)(top + total);
+}
+
 constexpr int kAppendTok = 8;   // tokens per CTA
 constexpr int kCopyThreads = 256;
 
@@ -289,6 +352,13 @@ cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int
   if (n_new == nullptr && new_offsets == nullptr) return cudaErrorInvalidValue;
   kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, new_offsets, B, page_ids_out,
                                                    page_ids_cap);
+  return cudaGetLastError();
+}
+
+cudaError_t kv_release_launch(const KvTableDev& t, const int64_t* users, int B,
+                              cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  kv_release_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, B);
   return cudaGetLastError();
 }
 

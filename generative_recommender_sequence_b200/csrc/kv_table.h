@@ -30,6 +30,9 @@ void kv_table_free_storage(KvTableDev* t);
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
                             int32_t* page_ids_out, int page_ids_cap, cudaStream_t stream,
                             const int64_t* new_offsets = nullptr);
+// Evicts whole users: their pages return to the free stack (see kv_table.cu).
+cudaError_t kv_release_launch(const KvTableDev& t, const int64_t* users, int B,
+                              cudaStream_t stream);
 // k_new / v_new rows are src_row_elems elements apart (0: H * d, packed rows).
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
                              const void* v_new, const int64_t* new_offsets, int B, int max_new,

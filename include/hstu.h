@@ -155,6 +155,21 @@ HSTU_API hstu_status hstu_kv_alloc(hstu_kv_table* t, const int64_t* users, const
                           cudaStream_t stream);
 
 /*
+ * Eviction of whole users (section "What the workflow combines" of the page
+ * cited above: older users are evicted LRU-style when the cache is full; the
+ * choice of users is the caller's).  Every page of each listed user returns to
+ * the free stack - users in the order listed, each user's pages from its last
+ * to its first, so its first page ends on top - and its cached length becomes
+ * 0.  users: [B] device, unique.  The page bytes are not cleared.  Duplicate
+ * or out-of-range users leave the table unchanged and record
+ * HSTU_ERR_INVALID_ARG in the status word.  To keep a user's K/V (host tier),
+ * gather it with hstu_kv_lookup first; to bring it back, hstu_kv_alloc then
+ * hstu_kv_append.
+ */
+HSTU_API hstu_status hstu_kv_release(hstu_kv_table* t, const int64_t* users, int32_t B,
+                                     cudaStream_t stream);
+
+/*
  * Append: token r of user users[b] (rows new_offsets[b] .. new_offsets[b+1]-1
  * of k_new / v_new, [T_new, H, d] in the table dtype) goes to page
  * list[len / page_size], slot len % page_size, then len grows.  Pages must

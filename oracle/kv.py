@@ -19,6 +19,11 @@ The pages give only the operation names.  The readings taken here:
   slot ``len_u % page_size``; then ``len_u`` grows by one;
 * ``lookup``: cached length per user, the user's page list padded with -1, and
   optionally a jagged copy of the cached K/V.
+* ``release(users)`` (eviction of whole users): every page of each listed user
+  goes back on the free stack - users in the order listed, each user's pages
+  from its last to its first, so its first page ends on top - and the user's
+  length and page list become empty; duplicate or out-of-range users leave the
+  table unchanged (INVALID_ARG).  The page bytes stay as they were.
 Element values are stored as raw bit patterns (uint16 for bf16, uint32 for
 fp32), so comparisons with the GPU pool are byte-exact.
 """
@@ -108,6 +113,18 @@ class KVTableOracle:
                 self.pool[page, 0, :, slot, :] = kb[t]
                 self.pool[page, 1, :, slot, :] = vb[t]
                 self.length[u] += 1
+        return OK
+
+    def release(self, users):
+        """Evict whole users: their pages return to the free stack."""
+        users = self._check_users(users)
+        if users is None:
+            return INVALID_ARG
+        for u in users:
+            for p in reversed(self.pages[u]):
+                self.stack.append(p)
+            self.pages[u] = []
+            self.length[u] = 0
         return OK
 
     def lookup(self, users, max_pages, gather=True):

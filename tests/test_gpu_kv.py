@@ -159,3 +159,58 @@ def test_kv_device_errors_leave_table_unchanged():
     t.lookup(dev(np.array([2], np.int64)), lens)
     assert lens.item() == 0
     t.close()
+
+
+def test_kv_release_bit_exact_through_later_allocations():
+    """Evictions interleaved with alloc / append: the page ids every later alloc
+    returns (which depend on the free-stack order release leaves) and the final
+    lookups and pool bytes match the oracle."""
+    import generative_recommender_sequence_b200 as hstu
+    rng = np.random.default_rng(3)
+    n_pages, H, d, U = 120, 4, 128, 10
+    order = rng.permutation(n_pages)
+    t = hstu.KVTable(n_pages, H, d, max_users=U, max_pages_per_user=64, free_order=order)
+    ref = KVTableOracle(n_pages, 32, H, d, U, 64, order)
+    for step in range(24):
+        B = int(rng.integers(1, 5))
+        users = rng.permutation(U)[:B]
+        if rng.random() < 0.35:
+            t.release(dev(users.astype(np.int64)))
+            assert t.status() == OK
+            assert ref.release(users.tolist()) == OK
+            continue
+        n = rng.integers(0, 120, size=B)
+        ids = torch.full((256,), -7, dtype=torch.int32, device="cuda")
+        t.alloc(dev(users.astype(np.int64)), dev(n.astype(np.int64)), page_ids_out=ids)
+        status = t.status()
+        rs, rpages = ref.alloc(users.tolist(), n.tolist())
+        assert status == rs
+        if rs != OK:
+            continue
+        assert ids.cpu().numpy()[: len(rpages)].tolist() == rpages
+        kv = workloads._as_storage(rng.standard_normal((2, int(n.sum()), H, d)).astype(np.float32), "bf16")
+        off = workloads.offsets_from_lengths(n)
+        t.append(dev(users.astype(np.int64)), storage(kv[0], "bf16"), storage(kv[1], "bf16"),
+                 dev(off), int(max(n.max(), 1)))
+        assert t.status() == OK
+        assert ref.append(users.tolist(), kv[0], kv[1], off) == OK
+    users = np.arange(U)
+    rl, rt, rk, rv = ref.lookup(users.tolist(), 64)
+    lens = torch.empty(U, dtype=torch.int64, device="cuda")
+    table = torch.empty((U, 64), dtype=torch.int32, device="cuda")
+    out_off = workloads.offsets_from_lengths(rl)
+    ko = torch.empty((max(int(out_off[-1]), 1), H, d), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    t.lookup(dev(users.astype(np.int64)), lens, table, ko, vo, dev(out_off), int(max(rl.max(), 1)))
+    assert np.array_equal(lens.cpu().numpy(), rl) and np.array_equal(table.cpu().numpy(), rt)
+    T = int(out_off[-1])
+    assert np.array_equal(ko[:T].cpu().view(torch.int16).numpy().view(np.uint16), rk)
+    assert np.array_equal(vo[:T].cpu().view(torch.int16).numpy().view(np.uint16), rv)
+    # duplicate users: rejected on the device, table unchanged
+    before = t.storage()
+    t.release(dev(np.array([1, 1], np.int64)))
+    assert t.status() == INVALID_ARG
+    lens2 = torch.empty(U, dtype=torch.int64, device="cuda")
+    t.lookup(dev(users.astype(np.int64)), lens2)
+    assert np.array_equal(lens2.cpu().numpy(), rl) and t.storage() == before
+    t.close()

@@ -168,3 +168,41 @@ def test_kv_errors_leave_table_unchanged():
     kv = np.zeros((5, 1, 2), np.float32)
     assert t.append([0], kv, kv, [0, 5]) == INVALID_ARG   # only 4 slots reserved
     assert t.length[0] == 0
+
+
+def test_kv_release_hand_example():
+    # free order 0..5 (top = 5); pages of 4 tokens
+    t = KVTableOracle(6, 4, 1, 2, 3, 8, [0, 1, 2, 3, 4, 5])
+    assert t.alloc([0, 1], [9, 2]) == (OK, [5, 4, 3, 2])
+    assert t.pages[0] == [5, 4, 3] and t.pages[1] == [2] and t.stack == [0, 1]
+    # user 1 first, then user 0; each user's pages go back last to first
+    assert t.release([1, 0]) == OK
+    assert t.stack == [0, 1, 2, 3, 4, 5]
+    assert t.pages[0] == [] and t.pages[1] == [] and t.length[0] == 0
+    # the next user gets user 0's first pages back, in the same order
+    assert t.alloc([2], [5]) == (OK, [5, 4])
+
+
+def test_kv_release_errors_and_accounting():
+    t = KVTableOracle(6, 4, 1, 2, 3, 8, [0, 1, 2, 3, 4, 5])
+    assert t.alloc([0], [6])[0] == OK
+    before = (list(t.stack), [list(p) for p in t.pages], list(t.length))
+    assert t.release([0, 0]) == INVALID_ARG
+    assert t.release([3]) == INVALID_ARG
+    assert (t.stack, t.pages, t.length) == before
+    # random alloc / append / release sequences keep every page exactly once
+    rng = np.random.default_rng(8)
+    t = KVTableOracle(64, 4, 1, 2, 6, 64, rng.permutation(64))
+    for _ in range(40):
+        users = rng.permutation(6)[:rng.integers(1, 4)].tolist()
+        if rng.random() < 0.4:
+            assert t.release(users) == OK
+            assert all(t.length[u] == 0 and t.pages[u] == [] for u in users)
+        else:
+            n = rng.integers(0, 9, size=len(users))
+            if t.alloc(users, n)[0] == OK:
+                kv = np.zeros((int(n.sum()), 1, 2), np.float32)
+                assert t.append(users, kv, kv, offsets_from_lengths(n)) == OK
+        held = [p for u in range(6) for p in t.pages[u]]
+        assert len(held) + t.n_free == 64 and set(held).isdisjoint(t.stack)
+        assert all(len(t.pages[u]) == -(-t.length[u] // 4) for u in range(6))
