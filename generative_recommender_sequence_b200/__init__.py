@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import (HSTU_BF16, HSTU_ERR_INVALID_ARG, HSTU_F32, HSTU_MASK_CANDIDATES,
                    HSTU_MASK_CAUSAL_SUFFIX, HstuError, HstuRab, check, declared_symbols, load)
 
-__all__ = ["attn_fwd", "attn_cached_fwd", "KVTable", "block_fwd", "block_cached_step",
+__all__ = ["attn_fwd", "attn_cached_fwd", "KVTable", "UserMap", "block_fwd", "block_cached_step",
            "block_cached_workspace_size", "HstuError", "load",
            "declared_symbols", "device_check", "last_device_error",
            "HSTU_MASK_CANDIDATES", "HSTU_MASK_CAUSAL_SUFFIX"]
@@ -159,6 +159,48 @@ class KVTable:
     def workspace_size(self, B: int, total_q: int, max_q: int, max_cached: int, mask_mode: int) -> int:
         return self.lib.hstu_attn_cached_workspace_size(self.handle, B, total_q, max_q, max_cached,
                                                         mask_mode)
+
+
+class UserMap:
+    """Sparse int64 user ids -> dense KV-table slots (hstu_user_map_* in include/hstu.h)."""
+
+    def __init__(self, n_slots: int, free_order: Optional[Sequence[int]] = None):
+        self.lib = load()
+        self.n_slots = n_slots
+        handle = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            arr = (ctypes.c_int32 * n_slots)(*[int(x) for x in free_order])
+            order = ctypes.cast(arr, ctypes.c_void_p)
+        check("hstu_user_map_create", self.lib.hstu_user_map_create(n_slots, order, ctypes.byref(handle)))
+        self.handle = handle
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.hstu_user_map_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def lookup(self, ids, insert: bool = True, out=None, stream=None) -> torch.Tensor:
+        _need_cuda(ids, out)
+        if out is None:
+            out = torch.empty(ids.numel(), dtype=torch.int64, device=ids.device)
+        check("hstu_user_map_lookup", self.lib.hstu_user_map_lookup(
+            self.handle, _ptr(ids), ids.numel(), 1 if insert else 0, _ptr(out), _stream(stream)))
+        return out
+
+    def erase(self, ids, stream=None):
+        _need_cuda(ids)
+        check("hstu_user_map_erase", self.lib.hstu_user_map_erase(self.handle, _ptr(ids), ids.numel(),
+                                                                  _stream(stream)))
+
+    def status(self, stream=None) -> int:
+        return self.lib.hstu_user_map_status(self.handle, _stream(stream))
 
 
 def attn_cached_fwd(table: KVTable, users, q, q_offsets, max_q: int, max_cached: int,

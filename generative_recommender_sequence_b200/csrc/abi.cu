@@ -15,6 +15,7 @@
 #include "attn.h"
 #include "block.h"
 #include "kv_table.h"
+#include "user_map.h"
 
 // Device error word written by kernels whose bounded waits ran out.
 __device__ int g_hstu_device_error;
@@ -553,6 +554,74 @@ hstu_status hstu_block_cached_step(hstu_kv_table* const* tables, int32_t n_layer
       hstu::block_cached_step_launch(p, workspace, ws_bytes, device_error_word(), stream);
   if (e == cudaErrorNotSupported) return HSTU_ERR_UNSUPPORTED;
   return from_cuda(e);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- user-id map
+struct hstu_user_map {
+  hstu::UserMapDev dev;
+};
+
+extern "C" {
+
+hstu_status hstu_user_map_create(int32_t n_slots, const int32_t* host_free_order,
+                                 hstu_user_map** out_map) {
+  if (!out_map || n_slots <= 0 || n_slots > (1 << 28)) return HSTU_ERR_INVALID_ARG;
+  *out_map = nullptr;
+  if (host_free_order) {
+    std::vector<char> seen((size_t)n_slots, 0);
+    for (int32_t i = 0; i < n_slots; ++i) {
+      const int32_t x = host_free_order[i];
+      if (x < 0 || x >= n_slots || seen[x]) return HSTU_ERR_INVALID_ARG;
+      seen[x] = 1;
+    }
+  }
+  hstu_user_map* m = new (std::nothrow) hstu_user_map();
+  if (!m) return HSTU_ERR_CUDA;
+  if (hstu::user_map_alloc(&m->dev, n_slots, host_free_order) != cudaSuccess) {
+    hstu::user_map_free(&m->dev);
+    delete m;
+    return HSTU_ERR_CUDA;
+  }
+  *out_map = m;
+  return HSTU_OK;
+}
+
+void hstu_user_map_destroy(hstu_user_map* m) {
+  if (!m) return;
+  hstu::user_map_free(&m->dev);
+  delete m;
+}
+
+hstu_status hstu_user_map_lookup(hstu_user_map* m, const int64_t* ids, int32_t B, int32_t insert,
+                                 int64_t* slots_out, cudaStream_t stream) {
+  if (!m || B < 0 || B > 65536) return HSTU_ERR_INVALID_ARG;
+  if (B == 0) return HSTU_OK;
+  if (!ids || !slots_out) return HSTU_ERR_INVALID_ARG;
+  return from_cuda(hstu::user_map_lookup_launch(m->dev, ids, B, insert != 0, slots_out, stream));
+}
+
+hstu_status hstu_user_map_erase(hstu_user_map* m, const int64_t* ids, int32_t B,
+                                cudaStream_t stream) {
+  if (!m || B < 0) return HSTU_ERR_INVALID_ARG;
+  if (B == 0) return HSTU_OK;
+  if (!ids) return HSTU_ERR_INVALID_ARG;
+  return from_cuda(hstu::user_map_erase_launch(m->dev, ids, B, stream));
+}
+
+hstu_status hstu_user_map_status(hstu_user_map* m, cudaStream_t stream) {
+  if (!m) return HSTU_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, m->dev.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (v != 0) {
+    const int32_t z = 0;
+    if (cudaMemcpy(m->dev.status, &z, sizeof(z), cudaMemcpyHostToDevice) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+  }
+  return (hstu_status)v;
 }
 
 }  // extern "C"

@@ -301,6 +301,35 @@ HSTU_API size_t hstu_block_cached_workspace_size(hstu_kv_table* const* tables, i
                                                  int32_t max_cand, int32_t max_cached,
                                                  int32_t d_model, int32_t H, int32_t dh);
 
+/*
+ * Sparse user-id -> dense slot map ("How Generative Recommenders Are Redefining
+ * RecSys at Scale", section "Dynamic embedding": sparse ids are hashed onto
+ * dense storage rows).  The slots (0 .. n_slots-1) name users of a KV table
+ * (max_users = n_slots): pass the slots_out array as its `users`.
+ *
+ * create: slots start free on a LIFO stack initialised from host_free_order (a
+ *   permutation of 0..n_slots-1, top = LAST element; NULL = 0..n_slots-1).
+ * lookup: ids [B] int64 device, each >= 0; slots_out [B] int64 device.  A
+ *   known id gets its slot.  With insert != 0 unknown ids take slots from the
+ *   top of the stack in the order listed (a repeated id shares the slot of its
+ *   first occurrence); with insert == 0 they get -1.  A negative id, or too
+ *   few free slots for the call's new ids, leaves the map unchanged, writes -1
+ *   everywhere and records HSTU_ERR_INVALID_ARG / HSTU_ERR_OUT_OF_PAGES (no
+ *   free slot) in the map's status word.  B <= 65536.
+ * erase: the listed ids' slots return to the stack in the order listed;
+ *   unknown ids are ignored.  Pair it with hstu_kv_release of the same slots.
+ * status: synchronises the stream, returns and clears the device error.
+ */
+typedef struct hstu_user_map hstu_user_map;
+HSTU_API hstu_status hstu_user_map_create(int32_t n_slots, const int32_t* host_free_order,
+                                          hstu_user_map** out_map);
+HSTU_API void hstu_user_map_destroy(hstu_user_map* m);
+HSTU_API hstu_status hstu_user_map_lookup(hstu_user_map* m, const int64_t* ids, int32_t B,
+                                          int32_t insert, int64_t* slots_out, cudaStream_t stream);
+HSTU_API hstu_status hstu_user_map_erase(hstu_user_map* m, const int64_t* ids, int32_t B,
+                                         cudaStream_t stream);
+HSTU_API hstu_status hstu_user_map_status(hstu_user_map* m, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
