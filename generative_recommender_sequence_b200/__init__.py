@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import (HSTU_BF16, HSTU_ERR_INVALID_ARG, HSTU_F32, HSTU_MASK_CANDIDATES,
                    HSTU_MASK_CAUSAL_SUFFIX, HstuError, HstuRab, check, declared_symbols, load)
 
-__all__ = ["attn_fwd", "attn_cached_fwd", "KVTable", "UserMap", "block_fwd", "block_cached_step",
+__all__ = ["attn_fwd", "attn_cached_fwd", "attn_beam_decode", "KVTable", "UserMap", "block_fwd", "block_cached_step",
            "block_cached_workspace_size", "HstuError", "load",
            "declared_symbols", "device_check", "last_device_error",
            "HSTU_MASK_CANDIDATES", "HSTU_MASK_CAUSAL_SUFFIX"]
@@ -304,3 +304,27 @@ def block_cached_step(tables: Sequence["KVTable"], users, x, new_offsets, max_ne
         workspace.numel() * workspace.element_size(), _stream(stream))
     check("hstu_block_cached_step", st)
     return x
+
+
+def attn_beam_decode(table: KVTable, users, q, beam_offsets, max_beams: int, max_ctx: int, step: int,
+                     beam_k, beam_v, beam_parent=None, pos_table=None, scale: float = 1.0, out=None,
+                     workspace=None, stream=None) -> torch.Tensor:
+    """Beam decode attention at step `step` over the shared context in `table`
+    (hstu_attn_beam_decode in include/hstu.h).  beam_k / beam_v: [step+1, T_beam, H, 128]."""
+    _need_cuda(users, q, beam_offsets, beam_k, beam_v, beam_parent, out)
+    if out is None:
+        out = torch.empty_like(q)
+    T = q.shape[0]
+    B = users.numel()
+    need = load().hstu_attn_beam_decode_workspace_size(table.handle, B, T, int(max_beams),
+                                                      int(max_ctx), int(step))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rab = _rab(pos_table, None, None)
+    st = load().hstu_attn_beam_decode(
+        table.handle, _ptr(users), B, _ptr(q), _ptr(beam_offsets), T, int(max_beams), int(max_ctx),
+        int(step), _ptr(beam_k), _ptr(beam_v), _ptr(beam_parent), ctypes.byref(rab) if rab else None,
+        float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    check("hstu_attn_beam_decode", st)
+    return out

@@ -52,6 +52,9 @@ _SIGNATURES = {
     "hstu_kv_alloc": ([_P, _P, _P, _I32, _P, _I32, _P], _I32),
     "hstu_kv_append": ([_P, _P, _P, _P, _P, _I32, _I32, _P], _I32),
     "hstu_kv_release": ([_P, _P, _I32, _P], _I32),
+    "hstu_attn_beam_decode": ([_P, _P, _I32, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _F, _P,
+                               _P, _SZ, _P], _I32),
+    "hstu_attn_beam_decode_workspace_size": ([_P, _I32, _I64, _I32, _I32, _I32], _SZ),
     "hstu_user_map_create": ([_I32, _P, _P], _I32),
     "hstu_user_map_destroy": ([_P], None),
     "hstu_user_map_lookup": ([_P, _P, _I32, _I32, _P, _P], _I32),

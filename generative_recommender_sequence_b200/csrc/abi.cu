@@ -13,6 +13,7 @@
 
 #include "../../include/hstu.h"
 #include "attn.h"
+#include "beam_decode.h"
 #include "block.h"
 #include "kv_table.h"
 #include "user_map.h"
@@ -622,6 +623,74 @@ hstu_status hstu_user_map_status(hstu_user_map* m, cudaStream_t stream) {
       return HSTU_ERR_CUDA;
   }
   return (hstu_status)v;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- beam decode
+extern "C" {
+
+static bool beam_problem(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
+                         const int64_t* beam_offsets, int64_t total_beams, int32_t max_beams,
+                         int32_t max_ctx, int32_t step, const void* beam_k, const void* beam_v,
+                         const int32_t* beam_parent, const hstu_rab* rab, float scale, void* out,
+                         hstu::BeamDecodeProblem* p) {
+  p->table = t->dev;
+  p->users = users;
+  p->B = B;
+  p->q = q;
+  p->beam_offsets = beam_offsets;
+  p->total_beams = total_beams;
+  p->max_beams = max_beams;
+  p->max_ctx = max_ctx;
+  p->step = step;
+  p->beam_k = beam_k;
+  p->beam_v = beam_v;
+  p->beam_parent = beam_parent;
+  if (rab && rab->pos_table) {
+    p->pos_table = rab->pos_table;
+    p->n_pos = rab->n_pos_buckets;
+  }
+  p->scale = scale;
+  p->out = out;
+  return true;
+}
+
+size_t hstu_attn_beam_decode_workspace_size(hstu_kv_table* t, int32_t B, int64_t total_beams,
+                                            int32_t max_beams, int32_t max_ctx, int32_t step) {
+  if (!t || B < 0 || total_beams < 0 || max_beams < 0 || max_ctx < 0 || step < 0) return 0;
+  hstu::BeamDecodeProblem p;
+  beam_problem(t, nullptr, B, nullptr, nullptr, total_beams, max_beams, max_ctx, step, nullptr,
+               nullptr, nullptr, nullptr, 1.f, nullptr, &p);
+  return hstu::beam_decode_workspace_bytes(p, device_sm_count());
+}
+
+hstu_status hstu_attn_beam_decode(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
+                                  const int64_t* beam_offsets, int64_t total_beams,
+                                  int32_t max_beams, int32_t max_ctx, int32_t step,
+                                  const void* beam_k, const void* beam_v,
+                                  const int32_t* beam_parent, const hstu_rab* rab, float scale,
+                                  void* out, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  if (!t || B < 0 || total_beams < 0 || max_beams < 0 || max_ctx < 0 || step < 0)
+    return HSTU_ERR_INVALID_ARG;
+  if (t->dtype != HSTU_BF16 || t->dev.d != 128 || t->dev.H > 32) return HSTU_ERR_UNSUPPORTED;
+  if ((int64_t)(step + 1) * total_beams >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
+  if (!rab_ok(rab, false)) return HSTU_ERR_UNSUPPORTED;
+  if (B == 0 || total_beams == 0) return HSTU_OK;
+  if (!users || !q || !beam_offsets || !beam_k || !beam_v || !out || max_beams <= 0)
+    return HSTU_ERR_INVALID_ARG;
+  if (step > 0 && !beam_parent) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(beam_k) || !aligned16(beam_v))
+    return HSTU_ERR_INVALID_ARG;
+  hstu::BeamDecodeProblem p;
+  beam_problem(t, users, B, q, beam_offsets, total_beams, max_beams, max_ctx, step, beam_k, beam_v,
+               beam_parent, rab, scale, out, &p);
+  const size_t need = hstu::beam_decode_workspace_bytes(p, device_sm_count());
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return HSTU_ERR_INVALID_ARG;
+  const cudaError_t e = hstu::beam_decode_launch(p, workspace, ws_bytes, device_error_word(), stream);
+  if (e == cudaErrorNotSupported) return HSTU_ERR_UNSUPPORTED;
+  return from_cuda(e);
 }
 
 }  // extern "C"

@@ -35,11 +35,18 @@ struct AttnProblem {
   int max_q = 0;                      // bound on per-user query count
   int max_kv = 0;                     // bound on per-user key count
   bool f32 = false;                   // fp32 tensors (SIMT kernel only)
+  // candidate mode: candidates sit at position (cached length + q_pos_offset)
+  int q_pos_offset = 0;
+  // write the unscaled fp32 partial sums of every key split to the workspace
+  // and leave the reduction to the caller (no output, no split reduce)
+  bool partial_only = false;
 };
 
 // bf16, d == 128, tcgen05 path.  workspace: fp32 split partials (may be null if
 // split_bytes() == 0).
 size_t attn_sm100_workspace_bytes(const AttnProblem& p, int num_sms);
+// The key-split plan the launch uses: n_split slices of kps key tiles each.
+void attn_sm100_split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps);
 cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_bytes,
                               int* err_word, cudaStream_t stream);
 

@@ -132,6 +132,7 @@ struct KParams {
   const float* time_table;
   int n_time;
   const int64_t* ts;
+  int q_pos_offset;
   float scale;
   __nv_bfloat16* out;
   int64_t out_stride;
@@ -255,7 +256,7 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
   }
   int total;
   if (CAND) {
-    it.p0 = it.n_k;
+    it.p0 = it.n_k + P.q_pos_offset;
     it.n_main = (int)((it.n_k + BN - 1) / BN);
     total = it.n_main + 1;
   } else {
@@ -1149,7 +1150,7 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tkc, tvc, kp);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
-  if (e != cudaSuccess || kp.partial == nullptr) return e;
+  if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
   split_reduce_kernel<PAGED><<<(unsigned)p.total_q, 128, 0, stream>>>(kp, p.B);
   return cudaGetLastError();
 }
@@ -1187,10 +1188,14 @@ void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
 
 }  // namespace
 
+void attn_sm100_split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
+  split_plan(p, num_sms, n_split, kps);
+}
+
 size_t attn_sm100_workspace_bytes(const AttnProblem& p, int num_sms) {
   int ns, kps;
   split_plan(p, num_sms, &ns, &kps);
-  if (ns <= 1) return 0;
+  if (ns <= 1 && !p.partial_only) return 0;
   return (size_t)ns * (size_t)p.total_q * p.H * HD * sizeof(float);
 }
 
@@ -1232,11 +1237,12 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
   kp.n_time = p.time_table ? p.n_time : 1;
   kp.ts = p.ts;
   kp.scale = p.scale;
+  kp.q_pos_offset = p.q_pos_offset;
   kp.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   kp.out_stride = p.out_stride;
   kp.total_q = p.total_q;
   kp.err = err_word;
-  if (kp.n_split > 1) {
+  if (kp.n_split > 1 || p.partial_only) {
     const size_t need = attn_sm100_workspace_bytes(p, num_sms);
     if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
     kp.partial = reinterpret_cast<float*>(workspace);

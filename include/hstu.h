@@ -302,6 +302,37 @@ HSTU_API size_t hstu_block_cached_workspace_size(hstu_kv_table* const* tables, i
                                                  int32_t d_model, int32_t H, int32_t dh);
 
 /*
+ * Beam-search decode attention over a shared context ("How Generative
+ * Recommenders Are Redefining RecSys at Scale", section "Semantic ID-GR": a
+ * request's long context is shared by all its beams (ContextKV), each beam has
+ * a short decode history (BeamKV) and an ancestry (BeamPath)).  The attention
+ * is the HSTU one used everywhere in this library.  At decode step `step` = s,
+ * beam j of request b sits at position L_b + s (L_b = the request's cached
+ * context length in table t, user users[b]) and attends to the context tokens
+ * (positions 0 .. L_b-1), to the decode tokens of its ancestors at steps
+ * 0 .. s-1 (positions L_b + t) and to its own token:
+ *   out = scale * sum_j SiLU(q . k_j + rab(|p - p_j|)) v_j.
+ * q: [total_beams, H, 128] bf16 device, this step's beam queries; requests'
+ *   beams are jagged by beam_offsets ([B+1] device), the same rows every step.
+ * beam_k, beam_v: [s+1][total_beams][H][128] bf16 device, the decode tokens' K
+ *   and V of steps 0 .. s (row s = this step's own tokens).
+ * beam_parent: [s+1][total_beams] int32 device (may be NULL when s == 0):
+ *   beam_parent[t][r] = index, within its request, of the step t-1 beam that
+ *   row r of step t extends.  max_ctx: bound on L_b.
+ * rab: position table only.  workspace: >= hstu_attn_beam_decode_workspace_size.
+ */
+HSTU_API hstu_status hstu_attn_beam_decode(hstu_kv_table* t, const int64_t* users, int32_t B,
+                                           const void* q, const int64_t* beam_offsets,
+                                           int64_t total_beams, int32_t max_beams,
+                                           int32_t max_ctx, int32_t step, const void* beam_k,
+                                           const void* beam_v, const int32_t* beam_parent,
+                                           const hstu_rab* rab, float scale, void* out,
+                                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+HSTU_API size_t hstu_attn_beam_decode_workspace_size(hstu_kv_table* t, int32_t B,
+                                                     int64_t total_beams, int32_t max_beams,
+                                                     int32_t max_ctx, int32_t step);
+
+/*
  * Sparse user-id -> dense slot map ("How Generative Recommenders Are Redefining
  * RecSys at Scale", section "Dynamic embedding": sparse ids are hashed onto
  * dense storage rows).  The slots (0 .. n_slots-1) name users of a KV table
