@@ -357,6 +357,74 @@ class CachedServingPart:
         return res
 
 
+class BeamDecodePart:
+    """Beam-search decode attention (the pages' Semantic ID workload shape, on
+    synthetic inputs): 8 requests with 5000-token contexts in the paged table,
+    256 beams each, 3 decode steps; 4 heads of 128, bf16.  Per step: latency,
+    FLOP rate, and the bytes that must move (context K/V once, the beams' Q, K,
+    V and output) as a fraction of HBM bandwidth."""
+
+    def __init__(self, seed=77, B=8, L=5000, W=256, steps=3):
+        import torch
+        import generative_recommender_sequence_b200 as hstu
+        import workloads as W_
+        rng = np.random.default_rng(seed)
+        self.hstu, self.B, self.L, self.W, self.steps = hstu, B, L, W, steps
+        H, D = 4, 128
+        bf = lambda shape: W_.to_torch(W_._as_storage(rng.standard_normal(shape).astype(np.float32),
+                                                      "bf16"), "bf16").cuda()
+        n_pages = B * ((L + 31) // 32) + 4
+        self.table = hstu.KVTable(n_pages, H, D, max_users=B, max_pages_per_user=(L + 31) // 32 + 2)
+        self.users = torch.arange(B, dtype=torch.int64, device="cuda")
+        lens = torch.full((B,), L, dtype=torch.int64, device="cuda")
+        self.table.alloc(self.users, lens)
+        off = torch.arange(0, B * L + 1, L, dtype=torch.int64, device="cuda")
+        self.table.append(self.users, bf((B * L, H, D)), bf((B * L, H, D)), off, L)
+        T = B * W
+        self.q = bf((T, H, D))
+        self.bk, self.bv = bf((steps, T, H, D)), bf((steps, T, H, D))
+        par = np.zeros((steps, T), np.int32)
+        for t in range(1, steps):
+            par[t] = np.concatenate([rng.integers(0, W, size=W) for _ in range(B)])
+        self.parent = torch.as_tensor(par).cuda()
+        self.bo = torch.arange(0, T + 1, W, dtype=torch.int64, device="cuda")
+        self.pt = torch.as_tensor(rng.normal(0, 0.1, 16).astype(np.float32)).cuda()
+        self.out = torch.empty_like(self.q)
+        self.ws = torch.empty(max(1 << 20, hstu.load().hstu_attn_beam_decode_workspace_size(
+            self.table.handle, B, T, W, L, steps - 1)), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def run(self, s):
+        self.hstu.attn_beam_decode(self.table, self.users, self.q, self.bo, self.W, self.L, s,
+                                   self.bk[:s + 1], self.bv[:s + 1], self.parent[:s + 1] if s else None,
+                                   pos_table=self.pt, scale=1.0 / (self.L + self.steps), out=self.out,
+                                   workspace=self.ws)
+
+    def measure(self, flush_buf, hbm_peak, tf_peak, reps=5):
+        import torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        res = {}
+        T, F = self.B * self.W, 4 * 128
+        for s in range(self.steps):
+            self.run(s)
+            tot = 0.0
+            for _ in range(reps):
+                flush_buf.fill_(1)
+                e0.record(); self.run(s); e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1) / 1e3
+            t = tot / reps
+            flops = float(T) * (self.L + s + 1) * F * 4
+            bytes_ = float(self.B) * self.L * F * 2 * 2 + T * F * 2 * (3 + 2 * s + 1)
+            res[f"step_{s}"] = {"us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 2),
+                                "frac_of_bf16_peak": round(flops / t / 1e12 / tf_peak, 4),
+                                "gbs": round(bytes_ / t / 1e9, 1),
+                                "frac_of_hbm": round(bytes_ / t / 1e9 / hbm_peak, 4)}
+        if self.table.status() or self.hstu.last_device_error():
+            raise RuntimeError("device error in the beam decode measurement")
+        return res
+
+
 def run_gpu(args):
     import torch
     import workloads as W
@@ -450,6 +518,8 @@ def run_gpu(args):
             serving[f"layers_{n_layers}"] = part.measure(runs=5)
             del part
 
+    beam = {} if args.no_serving else BeamDecodePart().measure(flush_buf, hbm_peak, tf_peak)
+
     e2e = run_e2e(A, Bp, flush_buf, args) if rank == 0 else None
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
@@ -474,6 +544,7 @@ def run_gpu(args):
                                       "candidates_per_s": round(cand_per_s, 1),
                                       "hbm_gbs": round(b_gbs, 1), "frac_of_hbm": round(b_gbs / hbm_peak, 4)},
                 "cached_serving": serving,
+                "beam_decode": beam,
                 "jagged_bf16": {"ms": round(jt / jsteps * 1e3, 4),
                                 "tflops": round(J.flops * jsteps / jt / 1e12, 2),
                                 "frac_of_bf16_peak": round(J.flops * jsteps / jt / 1e12 / tf_peak, 4)},
