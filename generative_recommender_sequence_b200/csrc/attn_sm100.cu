@@ -64,10 +64,16 @@ constexpr uint32_t TM_SP = 128;    // three S/P buffers of 128 columns each
 constexpr int NSP = 3;
 // whether eligible launches use CTA pairs when HSTU_ATTN_CTA_PAIRS is unset
 constexpr bool kCtaPairsByDefault = false;
-// P (bf16 pairs) overwrites the first half of each pointwise warp's own 32 S
-// columns: keys [32 c, 32 c + 32) -> columns [32 c, 32 c + 16) of the buffer,
-// so the 16 keys of MMA k-step kk start at column 32 (kk / 2) + 8 (kk % 2).
-__host__ __device__ constexpr uint32_t p_col(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
+// P (bf16 pairs) overwrites the first half of each pointwise warp's own S
+// columns.  16 warps per tile (32 columns each): keys [32 c, 32 c + 32) ->
+// columns [32 c, 32 c + 16), so MMA k-step kk (16 keys) starts at column
+// 32 (kk / 2) + 8 (kk % 2).  Two pairs of warpgroups (64 columns per warp):
+// keys [64 c, 64 c + 64) -> columns [64 c, 64 c + 32), k-step kk at
+// 64 (kk / 4) + 8 (kk % 4).
+template <bool PW2>
+__host__ __device__ constexpr uint32_t p_col(int kk) {
+  return PW2 ? 64 * (kk >> 2) + 8 * (kk & 3) : 32 * (kk >> 1) + 8 * (kk & 1);
+}
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
@@ -77,7 +83,9 @@ constexpr uint32_t kIdescPV2 = idesc_bf16_f32(2 * BM, HD, true);
 
 constexpr int NTS = 4;              // key-timestamp ring depth
 constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
-constexpr int RROW = 64;            // position-bias row per pointwise warp (its 32 columns + 31)
+constexpr int kRrowQuarters = 64;   // position-bias row per pointwise warp: 32 columns + 31
+constexpr int kRrowPairs = 96;      // same for the two-pair layout: 64 columns + 31
+constexpr int RROW = kRrowPairs;
 
 // Key timestamps of one key tile, staged by warp 2: exact float offsets from
 // the user's first timestamp (when |offset| < 2^23 for every key), plus the
@@ -108,8 +116,10 @@ struct __align__(1024) Smem {
   uint64_t v_full[VST], v_empty[VST];
   // s_full per (pair, buffer) = tile index mod 6, so each pair waits every phase
   // of its own barriers in order; p_full / sp_empty have one in-order waiter
-  uint64_t s_full[NSP], p_full[NSP], sp_empty[NSP];
-  uint64_t o_full, o_empty;
+  // s_full: one per buffer (16-warp layout) or per (pair, buffer) = tile mod 6
+  // (two-pair layout), so each waiter sees every phase of its barriers in order
+  uint64_t s_full[2 * NSP], p_full[NSP], sp_empty[NSP];
+  uint64_t o_full[2], o_empty;  // o_full[1]: second pair of the two-pair layout
   uint64_t ts_full[NTS], ts_empty[NTS];
   uint64_t qts_full[2], qts_empty[2];
   uint64_t mma_done, mma_done2;
@@ -408,7 +418,7 @@ __device__ __forceinline__ void pw_chunk_any(const uint32_t (&sv)[16], uint32_t 
 }
 
 // ------------------------------------------------------------ the kernel
-template <bool PAGED, bool CAND, bool PAIR>
+template <bool PAGED, bool CAND, bool PAIR, bool PW2>
 __global__ void __launch_bounds__(kThreads, 1)
     hstu_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -419,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
   static_assert(!(PAIR && CAND), "CTA pairs serve the causal path only");
+  static_assert(!(PAIR && PW2), "CTA pairs use the 16-warp pointwise layout");
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   // rank in the CTA pair (0 issues the pair's MMAs and owns the shared barriers)
@@ -457,17 +468,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.v_full[i]), 1);
       mbar_init(smem_u32(&sm.v_empty[i]), 1);
     }
-    // P written / O drained: the 16 pointwise warps, of each CTA of a pair
+    // P written / O drained: the warps that handle a tile (16, or one pair of
+    // 8 in the two-pair layout), of each CTA of a CTA pair
+    constexpr uint32_t kTileWarps = PW2 ? 8 : (PAIR ? 32 : 16);
+    for (int i = 0; i < 2 * NSP; ++i) mbar_init(smem_u32(&sm.s_full[i]), 1);
     for (int i = 0; i < NSP; ++i) {
-      mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.p_full[i]), PAIR ? 32 : 16);
+      mbar_init(smem_u32(&sm.p_full[i]), kTileWarps);
       mbar_init(smem_u32(&sm.sp_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.o_empty), PAIR ? 32 : 16);
+    mbar_init(smem_u32(&sm.o_full[0]), 1);
+    mbar_init(smem_u32(&sm.o_full[1]), 1);
+    mbar_init(smem_u32(&sm.o_empty), kTileWarps);
     for (int i = 0; i < NTS; ++i) {
       mbar_init(smem_u32(&sm.ts_full[i]), 1);
-      mbar_init(smem_u32(&sm.ts_empty[i]), 16);
+      mbar_init(smem_u32(&sm.ts_empty[i]), PW2 ? 8 : 16);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.qts_full[i]), 1);
@@ -687,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             commit<PAIR>(smem_u32(&sm.k_empty[slot]));
-            commit<PAIR>(smem_u32(&sm.s_full[sb]));
+            commit<PAIR>(smem_u32(&sm.s_full[PW2 ? g % (2 * NSP) : sb]));
             if (i == nt - 1) commit<PAIR>(smem_u32(&sm.q_empty[qs]));
           }
         } else {
@@ -708,16 +722,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               // (a CTA of a pair holds one 64-column half: the same layout)
               const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
               if (PAIR)
-                umma_ts_pair(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV2,
+                umma_ts_pair(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col<PW2>(kk), bdesc, kIdescPV2,
                              (i == 0 && kk == 0) ? 0u : 1u);
               else
-                umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col(kk), bdesc, kIdescPV,
+                umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col<PW2>(kk), bdesc, kIdescPV,
                         (i == 0 && kk == 0) ? 0u : 1u);
             }
             commit<PAIR>(smem_u32(&sm.v_empty[slot]));
             commit<PAIR>(smem_u32(&sm.sp_empty[pb]));
           }
-          if (ok) commit<PAIR>(smem_u32(&sm.o_full));
+          // two-pair layout: the pair that took the item's last key tile runs its epilogue
+          if (ok) commit<PAIR>(smem_u32(&sm.o_full[PW2 ? (g - 1) & 1 : 0]));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -813,6 +828,231 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok && lane == 0) record_timeout(P, sm);
     }
+  } else if (PW2 && warp >= 4) {
+    // =============================================== pointwise + epilogue (two pairs)
+    // 16 warps: key tiles alternate between two pairs of warpgroups; within a
+    // pair, warpgroup `chalf` takes score columns [64 chalf, 64 chalf + 64).
+    const int pwi = warp - 4;                       // 0..15
+    const int wg = pwi >> 3;                        // tile parity handled
+    const int chalf = (pwi >> 2) & 1;               // column half of the tile
+    const int sub = warp & 3;                       // TMEM lane quarter
+    const int r = sub * 32 + lane;                  // tile row owned by this thread
+    const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+    const bool use_time = P.time_table != nullptr && !PAGED && !CAND;
+    const bool use_pos = P.pos_table != nullptr;
+    float* rrow = sm.rrow[pwi];
+    const float self_rab = sm.pos_ext[0];
+    // last position bucket this thread read, and its bias (tiles far from the
+    // diagonal keep the same bucket for long runs, so the shared table is
+    // rarely touched on the constant-row path)
+    int pb_idx = -1;
+    float pb_val = 0.f;
+    Sched<PAIR ? 2 * BM : BM> sc;
+    sc.init(sm.m_q, P.B, HS, lane);
+    uint32_t qi = 0, g = 0, my_epi = 0;
+    bool ok = true;
+    for (long long rnd = 0; ok; ++rnd) {
+      const long long t = snake_item<PAIR>(rnd);
+      int b, m, rem;
+      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+      if (it.t0 >= it.t1) continue;
+      // this row's query position (every candidate sits at the cached length)
+      const int64_t qp = CAND ? it.p0 : it.p0 + r;
+      long long tq_i = 0;
+      float tq1 = 1.f;
+      bool tq_exact = true;
+      const uint32_t qsl = qi & 1;
+      if (use_time) {  // this row's timestamp, staged by warp 2
+        ok = mbar_wait_warp(smem_u32(&sm.qts_full[qsl]), (qi >> 1) & 1);
+        if (!ok) break;
+        tq_i = sm.qts[qsl].i[r];
+        tq1 = sm.qts[qsl].f[r] + 1.f;
+        tq_exact = sm.qts[qsl].exact != 0;
+      }
+      for (int tile = it.t0; tile < it.t1 && ok; ++tile, ++g) {
+        if ((int)(g & 1) != wg) continue;
+        const uint32_t sb = g % NSP;
+        const bool cand_tile = CAND && tile == it.n_main;
+        const int64_t k0 = (int64_t)tile * BN;      // key position of column 0
+        // int32 tile-relative coordinates: query position minus k0, valid keys
+        const int qrel = (int)max64(min64(qp - k0, 1 << 30), -(1 << 30));
+        // lane 0 has the warp's smallest query position
+        const int64_t qp0 = CAND ? it.p0 : it.p0 + sub * 32;
+        const int qrel0 = (int)max64(min64(qp0 - k0, 1 << 30), -(1 << 30));
+        const int kend = (int)max64(min64(it.n_k - k0, BN), 0);
+        // offset of this warp's column half in its position-bias row
+        const int roff = chalf ? 0 : 64;
+        // element (row lane, column c) reads rbase[127 - c]
+        const int rshift = use_pos ? ((CAND ? 0 : lane) - roff) : 0;
+        const float* rtab = use_pos ? rrow : sm.pos_ext;  // zeros without a table
+        const uint32_t tslot = g % NTS;
+        bool time_fast = false;
+        if (use_time) {
+          ok = mbar_wait_warp(smem_u32(&sm.ts_full[tslot]), (g / NTS) & 1);
+          if (!ok) break;
+          time_fast = tq_exact && sm.ts[tslot].exact;
+        }
+        // Far from the diagonal a row's 64 columns usually share one position
+        // bucket (and, with sorted key timestamps, one time bucket): then the
+        // whole bias is one constant per row and is folded into the SiLU.
+        float crow = 0.f;
+        bool rowconst = false;
+        if (!cand_tile) {
+          const int cbase = 64 * chalf;
+          const int dmax = qrel - cbase, dmin = qrel - cbase - 63;
+          bool ok_row = dmin >= 0 || CAND;  // every column of both chunks visible
+          if (CAND) ok_row = cbase + 63 < kend;
+          if (use_pos) {
+            const int b_hi = min(31 - __clz(max(dmax, 0) + 1), kMaxRab - 1);
+            const int b_lo = min(31 - __clz(max(dmin, 0) + 1), kMaxRab - 1);
+            if (b_hi != pb_idx) {
+              pb_idx = b_hi;
+              pb_val = sm.pos_ext[b_hi];
+            }
+            ok_row = ok_row && (b_hi == b_lo || pb_val == sm.pos_ext[b_lo]);
+            crow = pb_val;
+          }
+          if (use_time) {
+            const TsSlot& ts = sm.ts[tslot];
+            long long d_hi = tq_i - ts.i[cbase], d_lo = tq_i - ts.i[cbase + 63];
+            d_hi = d_hi < 0 ? 0 : d_hi;
+            d_lo = d_lo < 0 ? 0 : d_lo;
+            const int t_hi = min(63 - __clzll(d_hi + 1), kMaxRab - 1);
+            const int t_lo = min(63 - __clzll(d_lo + 1), kMaxRab - 1);
+            ok_row = ok_row && ts.sorted && sm.time_ext[t_hi] == sm.time_ext[t_lo];
+            crow += sm.time_ext[t_hi];
+          }
+          rowconst = __all_sync(0xffffffffu, ok_row);
+        }
+        // position-bias row of this warp, only needed off the constant-row path:
+        // rrow[j] = position bias at delta qrel0 + j + roff - 127; this warp's
+        // columns need j in [0, 95)
+        if (use_pos && !cand_tile && !rowconst) {
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < kRrowPairs / 32; ++i) {
+            const int j = lane + 32 * i;
+            const int delta = max(qrel0 + j + roff - 127, 0);
+            rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
+          }
+          __syncwarp();
+        }
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // this warp's 64 S columns and, over their first half, its 32 P columns
+        const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
+        const uint32_t p_addr = s_addr;
+        const float hrow = 0.5f * crow;
+        // Two 16-column chunks per (rolled) iteration: chunk q + 1 loads while
+        // chunk q computes.  P of chunk q goes to columns [8q, 8q + 8), which
+        // only covers S chunks already loaded into registers.
+        uint32_t sa[16], sb2[16], pk[8];
+        tmem_ld16(s_addr, sa);
+        if (rowconst) {
+#pragma unroll 1
+          for (int q = 0; q < 4; q += 2) {
+            tmem_wait_ld();
+            reg_fence(sa);
+            tmem_ld16(s_addr + (q + 1) * 16, sb2);
+            silu_rowconst(sa, pk, hrow);
+            tmem_st8(p_addr + q * 8, pk);
+            tmem_wait_ld();
+            reg_fence(sb2);
+            if (q == 0) tmem_ld16(s_addr + 32, sa);
+            silu_rowconst(sb2, pk, hrow);
+            tmem_st8(p_addr + (q + 1) * 8, pk);
+          }
+        } else {
+          const int cb0 = chalf * 64;
+          const float* rl0 = rtab + (rshift + 127 - cb0);
+          const TsSlot& ts = sm.ts[use_time ? tslot : 0];
+          const int tmode = use_time ? (time_fast ? 1 : 2) : 0;
+#pragma unroll 1
+          for (int q = 0; q < 4; q += 2) {
+            tmem_wait_ld();
+            reg_fence(sa);
+            tmem_ld16(s_addr + (q + 1) * 16, sb2);
+            pw_chunk_any<CAND>(sa, pk, cb0 + q * 16, cand_tile, sub, qrel0, kend, tmode, rl0 - q * 16,
+                               qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
+            tmem_st8(p_addr + q * 8, pk);
+            tmem_wait_ld();
+            reg_fence(sb2);
+            if (q == 0) tmem_ld16(s_addr + 32, sa);
+            pw_chunk_any<CAND>(sb2, pk, cb0 + q * 16 + 16, cand_tile, sub, qrel0, kend, tmode,
+                               rl0 - q * 16 - 16, qrel, r, ts, tq1, tq_i, sm.time_ext, self_rab);
+            tmem_st8(p_addr + (q + 1) * 8, pk);
+          }
+        }
+        if (use_time) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.ts_empty[tslot]));
+        }
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.p_full[sb]));
+      }
+      if (!ok) break;
+      if (use_time) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.qts_empty[qsl]));
+      }
+      // ---- epilogue, by the pair that processed the item's last key tile (so
+      // the other pair can start the next item at once); this warp stores O
+      // columns [64 chalf, 64 chalf + 64) of its 32 rows.
+      if ((int)((g - 1) & 1) != wg) {
+        ++qi;
+        continue;
+      }
+      // each pair has its own o_full barrier and waits every one of its phases
+      // in order (a parity wait must never run two phases ahead or behind)
+      ok = mbar_wait_warp(smem_u32(&sm.o_full[wg]), my_epi & 1);
+      ++my_epi;
+      if (!ok) break;
+      tc_fence_after();
+      const bool row_ok = r < it.nvalid && it.q_row0 + r < P.total_q;
+      const int64_t row = it.q_row0 + r;
+#pragma unroll 1
+      for (int q = 0; q < 2; ++q) {
+        const int ocol = 64 * chalf + 32 * q;
+        uint32_t oa[32];
+        tmem_ld32(tmem + lane_addr + TM_O + ocol, oa);
+        tmem_wait_ld();
+        reg_fence(oa);
+        if (q == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.o_empty));
+        }
+        if (!row_ok) continue;
+        if (P.partial) {
+          float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
+                       it.h * HD + ocol;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            reinterpret_cast<float4*>(dst)[j / 4] =
+                make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
+                            __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+        } else {
+          __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + ocol;
+          const float sc2 = P.scale;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(oa[j]) * sc2, __uint_as_float(oa[j + 1]) * sc2);
+            u.y = pack_bf16x2(__uint_as_float(oa[j + 2]) * sc2, __uint_as_float(oa[j + 3]) * sc2);
+            u.z = pack_bf16x2(__uint_as_float(oa[j + 4]) * sc2, __uint_as_float(oa[j + 5]) * sc2);
+            u.w = pack_bf16x2(__uint_as_float(oa[j + 6]) * sc2, __uint_as_float(oa[j + 7]) * sc2);
+            reinterpret_cast<uint4*>(dst)[j / 8] = u;
+          }
+        }
+      }
+      ++qi;
+    }
+    if (!ok && lane == 0) record_timeout(P, sm);
   } else if (warp >= 4) {
     // =============================================== pointwise + epilogue
     // 16 warps share every key tile: warp (cq, sub) takes score columns
@@ -915,7 +1155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (use_pos && !cand_tile && !rowconst) {
           __syncwarp();
 #pragma unroll
-          for (int i = 0; i < RROW / 32; ++i) {
+          for (int i = 0; i < kRrowQuarters / 32; ++i) {
             const int j = lane + 32 * i;
             const int delta = max(qrel0 + j + roff - 127, 0);
             rrow[j] = sm.pos_ext[min(31 - __clz(delta + 1), kMaxRab - 1)];
@@ -969,7 +1209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- epilogue: this warp stores O columns [32 cq, 32 cq + 32) of its
       // 32 rows (every warp waits every phase of o_full in order)
-      ok = mbar_wait_warp(smem_u32(&sm.o_full), qi & 1);
+      ok = mbar_wait_warp(smem_u32(&sm.o_full[0]), qi & 1);
       if (!ok) break;
       tc_fence_after();
       const bool row_ok = r < it.nvalid && it.q_row0 + r < P.total_q;
@@ -1076,7 +1316,7 @@ __global__ void split_reduce_kernel(KParams P, int B) {
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-template <bool PAGED, bool CAND, bool PAIR>
+template <bool PAGED, bool CAND, bool PAIR, bool PW2 = false>
 cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items, int num_sms,
                         cudaStream_t stream) {
   CUtensorMap tq, tk, tv, tkc, tvc;
@@ -1103,7 +1343,7 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     tkc = tq;
     tvc = tq;
   }
-  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PAIR>;
+  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PAIR, PW2>;
   static bool attr_set[64] = {};
   static int max_pairs[64] = {};
   int dev = 0;
@@ -1258,8 +1498,10 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
   const long long items = (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
   if (p.paged) {
     if (p.mode == 1) return launch_impl<true, true, false>(p, kp, items, num_sms, stream);
+    // paged causal attention (the long-history path) runs the two-pair
+    // pointwise layout: measured faster there than 16 warps per tile
     return pair ? launch_impl<true, false, true>(p, kp, items, num_sms, stream)
-                : launch_impl<true, false, false>(p, kp, items, num_sms, stream);
+                : launch_impl<true, false, false, true>(p, kp, items, num_sms, stream);
   }
   return p.mode == 1 ? launch_impl<false, true, false>(p, kp, items, num_sms, stream)
                      : launch_impl<false, false, false>(p, kp, items, num_sms, stream);
