@@ -204,8 +204,13 @@ HSTU_API hstu_status hstu_kv_lookup(hstu_kv_table* t, const int64_t* users, int3
  *    last n_q = q_offsets[b+1]-q_offsets[b] cached tokens (n_q <= cached_len).
  * rab: only the position term (time_table must be NULL).
  * total_q = q_offsets[B] (rows of q, k_cand, v_cand, out); max_q / max_cached
- * bound the per-user query count / cached length (launch sizing).  workspace: device scratch of hstu_attn_cached_workspace_size()
- * bytes, 256-byte aligned (may be NULL when that size is 0).  bf16 needs d=128.
+ * bound the per-user query count / cached length (launch sizing).
+ * workspace: device scratch of hstu_attn_cached_workspace_size() bytes,
+ * 256-byte aligned (may be NULL when that size is 0).  It holds fp32 partial
+ * sums when the keys are split over several CTAs: always possible with
+ * candidates, and in causal-suffix mode when no user has more than 128 query
+ * rows (a few new tokens over a long cache); the split partials are reduced in
+ * a fixed order, so results do not depend on scheduling.  bf16 needs d=128.
  */
 HSTU_API hstu_status hstu_attn_cached_fwd(hstu_kv_table* t, const int64_t* users, int32_t B,
                                  const void* q, const void* k_cand, const void* v_cand,
