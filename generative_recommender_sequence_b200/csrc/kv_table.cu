@@ -37,17 +37,45 @@ __device__ __forceinline__ void set_status(int32_t* status, int code) {
 
 constexpr int kAllocThreads = 1024;
 
+// Inclusive prefix sum of one value per thread over a kAllocThreads block
+// (warp shuffles, then the warp totals): three barriers.  *total gets the sum.
+__device__ int64_t block_inclusive_scan(int64_t x, int64_t* s_warp, int64_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int64_t w = s_warp[lane];  // kAllocThreads / 32 == 32 warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) x += s_warp[warp - 1];
+  *total = s_warp[31];
+  __syncthreads();
+  return x;
+}
+
 // One CTA.  Phase 1: per-user demand and validation.  Phase 2: block-wide
 // exclusive scan of the demand in the order users are listed.  Phase 3: pop
 // pages from the top of the free stack (user 0 first).
 __global__ void __launch_bounds__(kAllocThreads)
     kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new,
                     const int64_t* new_offsets, int B, int32_t* page_ids_out, int page_ids_cap) {
-  __shared__ int64_t s_chunk[kAllocThreads];
+  __shared__ int64_t s_warp[32];
   __shared__ int s_bad;
   __shared__ int s_epoch;
-  __shared__ int64_t s_total;
   const int tid = threadIdx.x;
+  // read early: only alloc / release change it, and they are stream-ordered
+  const int64_t top = *t.free_top;
   if (tid == 0) {
     s_bad = 0;
     s_epoch = atomicAdd(t.alloc_calls, 1) + 1;
@@ -72,19 +100,9 @@ __global__ void __launch_bounds__(kAllocThreads)
     if (t.n_held[u] + need > t.max_ppu) atomicOr(&s_bad, 1);
     mysum += need;
   }
-  s_chunk[tid] = mysum;
-  __syncthreads();
-  // phase 2: inclusive scan of the per-thread sums (Hillis-Steele)
-  for (int off = 1; off < kAllocThreads; off <<= 1) {
-    const int64_t x = tid >= off ? s_chunk[tid - off] : 0;
-    __syncthreads();
-    s_chunk[tid] += x;
-    __syncthreads();
-  }
-  if (tid == kAllocThreads - 1) s_total = s_chunk[tid];
-  __syncthreads();
-  const int64_t total = s_total;
-  const int64_t top = *t.free_top;
+  // phase 2: inclusive scan of the per-thread sums
+  int64_t total;
+  const int64_t incl = block_inclusive_scan(mysum, s_warp, &total);
   if (s_bad) {
     if (tid == 0) set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
     return;
@@ -94,7 +112,7 @@ __global__ void __launch_bounds__(kAllocThreads)
     return;
   }
   // phase 3
-  int64_t pre = s_chunk[tid] - mysum;  // exclusive prefix of this thread's first user
+  int64_t pre = incl - mysum;  // exclusive prefix of this thread's first user
   for (int b = b0; b < b1; ++b) {
     const int64_t u = users[b];
     const int64_t n = n_new ? n_new[b] : new_offsets[b + 1] - new_offsets[b];
@@ -123,11 +141,11 @@ __global__ void __launch_bounds__(kAllocThreads)
 // unchanged and set the status word.
 __global__ void __launch_bounds__(kAllocThreads)
     kv_release_kernel(KvTableDev t, const int64_t* users, int B) {
-  __shared__ int64_t s_chunk[kAllocThreads];
+  __shared__ int64_t s_warp[32];
   __shared__ int s_bad;
   __shared__ int s_epoch;
-  __shared__ int64_t s_total;
   const int tid = threadIdx.x;
+  const int64_t top = *t.free_top;
   if (tid == 0) {
     s_bad = 0;
     s_epoch = atomicAdd(t.alloc_calls, 1) + 1;
@@ -146,23 +164,13 @@ __global__ void __launch_bounds__(kAllocThreads)
     if (atomicExch(&t.epoch[u], epoch) == epoch) atomicOr(&s_bad, 1);  // listed twice
     mysum += t.n_held[u];
   }
-  s_chunk[tid] = mysum;
-  __syncthreads();
-  for (int off = 1; off < kAllocThreads; off <<= 1) {
-    const int64_t x = tid >= off ? s_chunk[tid - off] : 0;
-    __syncthreads();
-    s_chunk[tid] += x;
-    __syncthreads();
-  }
-  if (tid == kAllocThreads - 1) s_total = s_chunk[tid];
-  __syncthreads();
-  const int64_t total = s_total;
-  const int64_t top = *t.free_top;
+  int64_t total;
+  const int64_t incl = block_inclusive_scan(mysum, s_warp, &total);
   if (s_bad || top + total > t.n_pages) {
     if (tid == 0) set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
     return;
   }
-  int64_t pre = s_chunk[tid] - mysum;
+  int64_t pre = incl - mysum;
   for (int b = b0; b < b1; ++b) {
     const int64_t u = users[b];
     const int held = t.n_held[u];
@@ -179,15 +187,18 @@ __global__ void __launch_bounds__(kAllocThreads)
   if (tid == 0) *t.free_top = (int32_t)(top + total);
 }
 
-constexpr int kAppendTok = 8;   // tokens per CTA
+// tokens per CTA: at H * d = 512 bf16 elements a token's K and V rows are 128
+// 16-byte vectors, so 256 threads copy two tokens with one vector each
+constexpr int kAppendTok = 2;
 constexpr int kCopyThreads = 256;
 
 // grid (chunks, B): CTA (c, b) copies tokens [c*kAppendTok, ...) of user b.
 // The length is read before any copy and advanced by the last CTA of the user.
 template <int ESZ>
 __global__ void __launch_bounds__(kCopyThreads)
-    kv_append_kernel(KvTableDev t, const int64_t* users, const uint8_t* k_new, const uint8_t* v_new,
-                     const int64_t* new_offsets, int64_t src_row_bytes) {
+    kv_append_kernel(KvTableDev t, const int64_t* __restrict__ users,
+                     const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
+                     const int64_t* __restrict__ new_offsets, int64_t src_row_bytes) {
   const int b = blockIdx.y;
   const int64_t u = users[b];
   const int64_t s = new_offsets[b], n = new_offsets[b + 1] - s;
