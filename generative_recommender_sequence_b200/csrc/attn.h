@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "launch.h"
+
 namespace hstu {
 
 // Where the keys/values of a (user, head) come from and which mask applies.

@@ -434,6 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   // rank in the CTA pair (0 issues the pair's MMAs and owns the shared barriers)
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  // dependent launch: the next kernel may start being scheduled; this one waits
+  // for the previous kernel (which may have written the KV table) to finish
+  pdl_launch_dependents();
+  pdl_wait();
 
   // ---- setup
   for (int b = tid; b <= P.B; b += kThreads) {
@@ -1268,6 +1272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // sum the valid splits in split order, scale, round to bf16.
 template <bool PAGED>
 __global__ void split_reduce_kernel(KParams P, int B) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t row = blockIdx.x;
   if (row >= P.total_q || row >= P.q_off[B]) return;
   // find the user of this row
@@ -1358,8 +1364,8 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
   if (!PAIR) {
     const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
     if (!cached && dev >= 0 && dev < 64) attr_set[dev] = true;
-    kern<<<grid, kThreads, smem_bytes(), stream>>>(tq, tk, tv, tkc, tvc, kp);
-    e = cudaGetLastError();
+    e = launch_dependent(kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq, tk, tv, tkc,
+                         tvc, kp);
   } else {
     // persistent CTA pairs: as many 2-CTA clusters as can be resident at once
     cudaLaunchConfig_t cfg = {};
@@ -1391,8 +1397,8 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
-  split_reduce_kernel<PAGED><<<(unsigned)p.total_q, 128, 0, stream>>>(kp, p.B);
-  return cudaGetLastError();
+  return launch_dependent(split_reduce_kernel<PAGED>, dim3((unsigned)p.total_q), dim3(128), 0, stream,
+                          kp, p.B);
 }
 
 // -1 when HSTU_ATTN_CTA_PAIRS is unset, else 0 / 1.

@@ -21,6 +21,7 @@
 
 #include "attn.h"
 #include "beam_decode.h"
+#include "sm100.cuh"
 
 namespace hstu {
 
@@ -54,6 +55,8 @@ __device__ __forceinline__ float silu(float x) { return x / (1.f + __expf(-x)); 
 
 // One CTA per beam row, one warp per head, 4 features per lane.
 __global__ void beam_path_kernel(BeamParams P) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t r = blockIdx.x;
   const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (r >= P.total_beams || h >= P.H) return;
@@ -182,8 +185,8 @@ cudaError_t beam_decode_launch(const BeamDecodeProblem& p, void* workspace, size
   bp.partial = static_cast<const float*>(workspace);
   attn_sm100_split_plan(a, device_sm_count(), &bp.n_split, &bp.kps);
   bp.out = static_cast<__nv_bfloat16*>(p.out);
-  beam_path_kernel<<<(unsigned)p.total_beams, 32 * p.table.H, 0, stream>>>(bp);
-  return cudaGetLastError();
+  return launch_dependent(beam_path_kernel, dim3((unsigned)p.total_beams), dim3(32 * p.table.H), 0,
+                          stream, bp);
 }
 
 }  // namespace hstu

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  pdl_wait();  // A (and, with the residual epilogue, the output) come from earlier kernels
   const int m_tiles = (P.M + GBM - 1) / GBM, n_tiles = P.N / GBN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = P.K / GBK;
@@ -226,6 +228,8 @@ __global__ void __launch_bounds__(256)
     ln_gate_kernel(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ u,
                    int64_t ldu, __nv_bfloat16* __restrict__ g, int64_t T, float eps) {
   constexpr int F = 512;
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -297,8 +301,7 @@ cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb,
   const int tiles = ((M + GBM - 1) / GBM) * (N / GBN);
   const int grid = std::max(1, std::min(tiles, device_sm_count()));
   GemmParams p{M, N, K, reinterpret_cast<__nv_bfloat16*>(out), ldo, err};
-  kern<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(), stream, ta, tb, p);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -348,9 +351,8 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
     a.max_q = a.max_kv = p.max_len;
     e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
     if (e != cudaSuccess) return e;
-    ln_gate_kernel<<<(unsigned)((p.T + 7) / 8), 256, 0, stream>>>(attn, uvqk, 4 * F, gate, p.T,
-                                                                  p.ln_eps);
-    e = cudaGetLastError();
+    e = launch_dependent(ln_gate_kernel, dim3((unsigned)((p.T + 7) / 8)), dim3(256), 0, stream,
+                         attn, uvqk, 4 * F, gate, p.T, p.ln_eps);
     if (e != cudaSuccess) return e;
     e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
                                   err_word, stream);
@@ -463,8 +465,8 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
       e = attn_sm100_launch(a, split_ws, split_bytes, err_word, stream);
       if (e != cudaSuccess) return e;
     }
-    ln_gate_kernel<<<(unsigned)((T + 7) / 8), 256, 0, stream>>>(attn, uvqk, 4 * F, gate, T, p.ln_eps);
-    e = cudaGetLastError();
+    e = launch_dependent(ln_gate_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, stream, attn,
+                         uvqk, 4 * F, gate, T, p.ln_eps);
     if (e != cudaSuccess) return e;
     e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
                                   err_word, stream);

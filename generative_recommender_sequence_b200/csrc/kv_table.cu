@@ -26,6 +26,8 @@
 #include <vector>
 
 #include "kv_table.h"
+#include "launch.h"
+#include "sm100.cuh"
 
 namespace hstu {
 
@@ -74,6 +76,8 @@ __global__ void __launch_bounds__(kAllocThreads)
   __shared__ int s_bad;
   __shared__ int s_epoch;
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   // read early: only alloc / release change it, and they are stream-ordered
   const int64_t top = *t.free_top;
   if (tid == 0) {
@@ -145,6 +149,8 @@ __global__ void __launch_bounds__(kAllocThreads)
   __shared__ int s_bad;
   __shared__ int s_epoch;
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t top = *t.free_top;
   if (tid == 0) {
     s_bad = 0;
@@ -199,6 +205,8 @@ __global__ void __launch_bounds__(kCopyThreads)
     kv_append_kernel(KvTableDev t, const int64_t* __restrict__ users,
                      const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
                      const int64_t* __restrict__ new_offsets, int64_t src_row_bytes) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y;
   const int64_t u = users[b];
   const int64_t s = new_offsets[b], n = new_offsets[b + 1] - s;
@@ -252,6 +260,8 @@ __global__ void __launch_bounds__(kCopyThreads)
     kv_lookup_kernel(KvTableDev t, const int64_t* users, int64_t* cached_len_out,
                      int32_t* page_table_out, int max_pages, uint8_t* k_out, uint8_t* v_out,
                      const int64_t* out_offsets) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y;
   const int64_t u = users[b];
   const bool valid_user = u >= 0 && u < t.max_users;
@@ -361,16 +371,14 @@ cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int
                             const int64_t* new_offsets) {
   if (B == 0 && page_ids_out == nullptr) return cudaSuccess;
   if (n_new == nullptr && new_offsets == nullptr) return cudaErrorInvalidValue;
-  kv_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, n_new, new_offsets, B, page_ids_out,
-                                                   page_ids_cap);
-  return cudaGetLastError();
+  return launch_dependent(kv_alloc_kernel, dim3(1), dim3(kAllocThreads), 0, stream, t, users, n_new,
+                          new_offsets, B, page_ids_out, page_ids_cap);
 }
 
 cudaError_t kv_release_launch(const KvTableDev& t, const int64_t* users, int B,
                               cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
-  kv_release_kernel<<<1, kAllocThreads, 0, stream>>>(t, users, B);
-  return cudaGetLastError();
+  return launch_dependent(kv_release_kernel, dim3(1), dim3(kAllocThreads), 0, stream, t, users, B);
 }
 
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
@@ -383,12 +391,10 @@ cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const vo
     return cudaErrorInvalidValue;
   dim3 grid((max_new + kAppendTok - 1) / kAppendTok, B);
   if (t.esize == 2)
-    kv_append_kernel<2><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 2);
-  else
-    kv_append_kernel<4><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 4);
-  return cudaGetLastError();
+    return launch_dependent(kv_append_kernel<2>, grid, dim3(kCopyThreads), 0, stream, t, users,
+                            (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 2);
+  return launch_dependent(kv_append_kernel<4>, grid, dim3(kCopyThreads), 0, stream, t, users,
+                          (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 4);
 }
 
 cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
@@ -399,14 +405,12 @@ cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
   const int chunks = k_out ? std::max(1, (max_len + kAppendTok - 1) / kAppendTok) : 1;
   dim3 grid(chunks, B);
   if (t.esize == 2)
-    kv_lookup_kernel<2><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, cached_len_out, page_table_out, max_pages, (uint8_t*)k_out, (uint8_t*)v_out,
-        out_offsets);
-  else
-    kv_lookup_kernel<4><<<grid, kCopyThreads, 0, stream>>>(
-        t, users, cached_len_out, page_table_out, max_pages, (uint8_t*)k_out, (uint8_t*)v_out,
-        out_offsets);
-  return cudaGetLastError();
+    return launch_dependent(kv_lookup_kernel<2>, grid, dim3(kCopyThreads), 0, stream, t, users,
+                            cached_len_out, page_table_out, max_pages, (uint8_t*)k_out,
+                            (uint8_t*)v_out, out_offsets);
+  return launch_dependent(kv_lookup_kernel<4>, grid, dim3(kCopyThreads), 0, stream, t, users,
+                          cached_len_out, page_table_out, max_pages, (uint8_t*)k_out,
+                          (uint8_t*)v_out, out_offsets);
 }
 
 }  // namespace hstu

@@ -213,6 +213,19 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel of the
+// stream still runs; it must call pdl_wait() before touching anything that
+// kernel writes.  pdl_launch_dependents() lets the next kernel start early.
+// Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs
 // A 2-CTA cluster shares one tcgen05.mma of M = 256: the even CTA (rank 0)
 // issues it, each CTA supplies half of A (its own 128 rows) and half of B (N/2
