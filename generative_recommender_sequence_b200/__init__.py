@@ -141,6 +141,16 @@ class KVTable:
                                      _ptr(new_offsets), users.numel(), int(max_new), _stream(stream))
         check("hstu_kv_append", st)
 
+    def step(self, users, k_new, v_new, new_offsets, max_new: int, cached_len_out=None,
+             page_table_out=None, stream=None):
+        """alloc + append + lookup rows of one serving step, all or nothing (hstu_kv_step)."""
+        _need_cuda(users, k_new, v_new, new_offsets, cached_len_out, page_table_out)
+        max_pages = 0 if page_table_out is None else page_table_out.shape[-1]
+        st = self.lib.hstu_kv_step(self.handle, _ptr(users), _ptr(k_new), _ptr(v_new), _ptr(new_offsets),
+                                   users.numel(), int(max_new), _ptr(cached_len_out),
+                                   _ptr(page_table_out), max_pages, _stream(stream))
+        check("hstu_kv_step", st)
+
     def release(self, users, stream=None):
         """Evict whole users: every page of each listed user returns to the free stack."""
         _need_cuda(users)

@@ -338,6 +338,21 @@ hstu_status hstu_kv_lookup(hstu_kv_table* t, const int64_t* users, int32_t B,
                                     k_out, v_out, out_offsets, max_len, stream));
 }
 
+hstu_status hstu_kv_step(hstu_kv_table* t, const int64_t* users, const void* k_new,
+                         const void* v_new, const int64_t* new_offsets, int32_t B, int32_t max_new,
+                         int64_t* cached_len_out, int32_t* page_table_out, int32_t max_pages,
+                         cudaStream_t stream) {
+  if (!t || B < 0 || max_new < 0 || max_pages < 0) return HSTU_ERR_INVALID_ARG;
+  if (B == 0) return HSTU_OK;
+  if (!users || !new_offsets) return HSTU_ERR_INVALID_ARG;
+  if (max_new > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return HSTU_ERR_INVALID_ARG;
+  if (page_table_out == nullptr) max_pages = 0;
+  if (B > 65535) return HSTU_ERR_UNSUPPORTED;
+  return from_cuda(kv_step_launch(t->dev, users, k_new, v_new, new_offsets, B, max_new,
+                                  cached_len_out, page_table_out, max_pages, stream));
+}
+
 static bool cached_problem(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
                            const void* k_cand, const void* v_cand, const int64_t* q_offsets,
                            int64_t total_q, int32_t max_q, int32_t max_cached, int32_t mask_mode,

@@ -434,30 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   // rank in the CTA pair (0 issues the pair's MMAs and owns the shared barriers)
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  // dependent launch: the next kernel may start being scheduled; this one waits
-  // for the previous kernel (which may have written the KV table) to finish
+  // dependent launch: the next kernel may start being scheduled.  Barrier
+  // initialisation, the descriptor prefetch and the TMEM allocation touch no
+  // global memory, so they overlap the previous kernel's tail; every global
+  // read comes after the wait for that kernel (which may have written the KV
+  // table or this kernel's inputs).
   pdl_launch_dependents();
-  pdl_wait();
-
-  // ---- setup
-  for (int b = tid; b <= P.B; b += kThreads) {
-    sm.m_q[b] = (int)P.q_off[b];
-    if (b == P.B) continue;
-    if (PAGED) {
-      // an out-of-range user id has no cached tokens (and no page list is read)
-      const int64_t u = P.users[b];
-      const bool known = u >= 0 && u < P.max_users;
-      sm.m_kv[b] = known ? (int)u : 0;
-      sm.m_nk[b] = known ? (int)P.lengths[u] : 0;
-    } else {
-      sm.m_kv[b] = (int)P.kv_off[b];
-      sm.m_nk[b] = (int)(P.kv_off[b + 1] - P.kv_off[b]);
-    }
-  }
-  for (int i = tid; i < kMaxRab; i += kThreads) {
-    sm.pos_ext[i] = P.pos_table ? P.pos_table[min(i, P.n_pos - 1)] : 0.f;
-    sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
-  }
   if (tid == 0) {
     sm.abort_flag = 0;
     for (int i = 0; i < QST; ++i) {
@@ -510,6 +492,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_alloc(smem_u32(&sm.tmem_base), 512);
       tmem_relinquish();
     }
+  }
+  pdl_wait();
+
+  // ---- setup
+  for (int b = tid; b <= P.B; b += kThreads) {
+    sm.m_q[b] = (int)P.q_off[b];
+    if (b == P.B) continue;
+    if (PAGED) {
+      // an out-of-range user id has no cached tokens (and no page list is read)
+      const int64_t u = P.users[b];
+      const bool known = u >= 0 && u < P.max_users;
+      sm.m_kv[b] = known ? (int)u : 0;
+      sm.m_nk[b] = known ? (int)P.lengths[u] : 0;
+    } else {
+      sm.m_kv[b] = (int)P.kv_off[b];
+      sm.m_nk[b] = (int)(P.kv_off[b + 1] - P.kv_off[b]);
+    }
+  }
+  for (int i = tid; i < kMaxRab; i += kThreads) {
+    sm.pos_ext[i] = P.pos_table ? P.pos_table[min(i, P.n_pos - 1)] : 0.f;
+    sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
   }
   tc_fence_before();
   __syncthreads();

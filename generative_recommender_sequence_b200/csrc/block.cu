@@ -64,8 +64,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // dependent launch: barrier set-up and the TMEM allocation overlap the
+  // previous kernel's tail; global memory is touched only after the wait
   pdl_launch_dependents();
-  pdl_wait();  // A (and, with the residual epilogue, the output) come from earlier kernels
   const int m_tiles = (P.M + GBM - 1) / GBM, n_tiles = P.N / GBN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = P.K / GBK;
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
   }
+  pdl_wait();  // A (and, with the residual epilogue, the output) come from earlier kernels
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -448,10 +450,8 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
     if (p.T_new > 0) {
       // the new tokens' K, V join this layer's cache, then they attend causally
       // over the cached history and themselves
-      e = kv_alloc_launch(t, p.users, nullptr, p.B, nullptr, 0, stream, p.new_offsets);
-      if (e != cudaSuccess) return e;
-      e = kv_append_launch(t, p.users, uvqk + 3 * F, uvqk + F, p.new_offsets, p.B, p.max_new, stream,
-                           4 * F);
+      e = kv_step_launch(t, p.users, uvqk + 3 * F, uvqk + F, p.new_offsets, p.B, p.max_new, nullptr,
+                         nullptr, 0, stream, 4 * F);
       if (e != cudaSuccess) return e;
       const AttnProblem a =
           cached_attention(p, t, false, uvqk, p.new_offsets, p.T_new, p.max_new, attn);

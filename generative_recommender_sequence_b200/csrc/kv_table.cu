@@ -18,6 +18,8 @@
 //               launch still gets a fresh epoch
 //   done        [max_users] int32: append chunk counters (always back to 0)
 //   status      first device-side error since the last status read
+//   step_done   CTAs of a one-launch serving step that finished (back to 0)
+//   step_ok     whether the alloc half of a two-launch serving step succeeded
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -71,7 +73,8 @@ __device__ int64_t block_inclusive_scan(int64_t x, int64_t* s_warp, int64_t* tot
 // pages from the top of the free stack (user 0 first).
 __global__ void __launch_bounds__(kAllocThreads)
     kv_alloc_kernel(KvTableDev t, const int64_t* users, const int64_t* n_new,
-                    const int64_t* new_offsets, int B, int32_t* page_ids_out, int page_ids_cap) {
+                    const int64_t* new_offsets, int B, int32_t* page_ids_out, int page_ids_cap,
+                    int32_t* ok_out, int64_t max_count) {
   __shared__ int64_t s_warp[32];
   __shared__ int s_bad;
   __shared__ int s_epoch;
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kAllocThreads)
   for (int b = b0; b < b1; ++b) {
     const int64_t u = users[b];
     const int64_t n = n_new ? n_new[b] : new_offsets[b + 1] - new_offsets[b];
-    if (u < 0 || u >= t.max_users || n < 0) {
+    if (u < 0 || u >= t.max_users || n < 0 || (max_count >= 0 && n > max_count)) {
       atomicOr(&s_bad, 1);
       continue;
     }
@@ -108,11 +111,17 @@ __global__ void __launch_bounds__(kAllocThreads)
   int64_t total;
   const int64_t incl = block_inclusive_scan(mysum, s_warp, &total);
   if (s_bad) {
-    if (tid == 0) set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
+    if (tid == 0) {
+      set_status(t.status, 1 /* HSTU_ERR_INVALID_ARG */);
+      if (ok_out) *ok_out = 0;
+    }
     return;
   }
   if (total > top) {
-    if (tid == 0) set_status(t.status, 2 /* HSTU_ERR_OUT_OF_PAGES */);
+    if (tid == 0) {
+      set_status(t.status, 2 /* HSTU_ERR_OUT_OF_PAGES */);
+      if (ok_out) *ok_out = 0;
+    }
     return;
   }
   // phase 3
@@ -135,7 +144,10 @@ __global__ void __launch_bounds__(kAllocThreads)
   if (page_ids_out)
     for (int64_t i = total + tid; i < page_ids_cap; i += kAllocThreads) page_ids_out[i] = -1;
   __syncthreads();
-  if (tid == 0) *t.free_top = (int32_t)(top - total);
+  if (tid == 0) {
+    *t.free_top = (int32_t)(top - total);
+    if (ok_out) *ok_out = 1;
+  }
 }
 
 // One CTA.  Releases every page of the listed users (eviction of whole users):
@@ -300,6 +312,205 @@ __global__ void __launch_bounds__(kCopyThreads)
   }
 }
 
+// One serving step: alloc + append + lookup rows, all or nothing.
+//
+// Small batches (B <= kStepMaxUsers) run as ONE launch of grid (chunks, B).
+// Every CTA reads the listed users' lengths and page counts and the free-stack
+// top at entry and re-derives the whole batch's allocation from them
+// (validation, per-user page demand, exclusive scan in listed order, pages
+// popped from the top of the stack), so all CTAs reach the same verdict and
+// the same page ids without waiting on each other.  CTA (c, b) copies tokens
+// [2c, 2c + 2) of user b into their slots; CTA (0, b) also writes user b's new
+// page-list entries and its lookup row.  None of the state read at entry is
+// written until every CTA has finished: the last CTA to finish (a grid-wide
+// counter) commits lengths, page counts and the stack top and resets the
+// counter.  An invalid batch or a lack of pages changes nothing (the lookup
+// rows then show the unchanged state) and records the status.
+//
+// Larger batches (PLAN = false) follow the alloc kernel, which records its
+// success in step_ok: the tokens are copied and the lengths advanced (last CTA
+// of each user) only when it succeeded; the lookup rows are written either way.
+constexpr int kStepMaxUsers = 64;
+
+template <int ESZ, bool PLAN>
+__global__ void __launch_bounds__(kCopyThreads)
+    kv_step_kernel(KvTableDev t, const int64_t* __restrict__ users,
+                   const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
+                   const int64_t* __restrict__ new_offsets, int B, int max_new,
+                   int64_t src_row_bytes, int64_t* __restrict__ cached_len_out,
+                   int32_t* __restrict__ page_table_out, int max_pages) {
+  __shared__ int64_t s_u[kStepMaxUsers];
+  __shared__ int64_t s_len[kStepMaxUsers];
+  __shared__ int s_held[kStepMaxUsers];
+  __shared__ int s_need[kStepMaxUsers];
+  __shared__ int s_pre[kStepMaxUsers + 1];
+  __shared__ int64_t s_top;
+  __shared__ int s_bad, s_ok, s_last;
+  const int tid = threadIdx.x, b = blockIdx.y;
+  pdl_launch_dependents();
+  pdl_wait();
+  int64_t u, len, top = 0;
+  int held, need = 0, pre = 0;
+  const int64_t n = new_offsets[b + 1] - new_offsets[b];
+  if (PLAN) {
+    if (tid == 0) {
+      s_bad = 0;
+      s_top = *t.free_top;
+    }
+    if (tid < kStepMaxUsers) s_need[tid] = 0;
+    __syncthreads();
+    if (tid < B) {
+      const int64_t ui = users[tid];
+      const int64_t ni = new_offsets[tid + 1] - new_offsets[tid];
+      int64_t li = 0;
+      int hi = 0, nd = 0;
+      if (ui < 0 || ui >= t.max_users) {
+        atomicOr(&s_bad, 1);
+      } else {
+        // read for every known user: a failed step still reports its state
+        li = t.lengths[ui];
+        hi = t.n_held[ui];
+        if (ni < 0 || ni > max_new) {
+          atomicOr(&s_bad, 1);
+        } else {
+          const int64_t want = (li + ni + t.page_size - 1) / t.page_size;
+          const int64_t d = want > hi ? want - hi : 0;
+          if (hi + d > t.max_ppu)
+            atomicOr(&s_bad, 1);
+          else
+            nd = (int)d;
+        }
+      }
+      s_u[tid] = ui;
+      s_len[tid] = li;
+      s_held[tid] = hi;
+      s_need[tid] = nd;
+    }
+    __syncthreads();
+    if (tid < B) {
+      for (int j = 0; j < tid; ++j)
+        if (s_u[j] == s_u[tid]) {  // listed twice
+          atomicOr(&s_bad, 1);
+          break;
+        }
+    }
+    if (tid < 32) {
+      // exclusive scan of the demand in listed order: lane l holds users l, 32 + l
+      int a = s_need[tid], c = s_need[32 + tid];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, a, o);
+        const int yc = __shfl_up_sync(0xffffffffu, c, o);
+        if (tid >= o) {
+          a += ya;
+          c += yc;
+        }
+      }
+      const int ta = __shfl_sync(0xffffffffu, a, 31);
+      s_pre[tid + 1] = a;
+      s_pre[tid + 33] = c + ta;
+      if (tid == 0) s_pre[0] = 0;
+    }
+    __syncthreads();
+    top = s_top;
+    const bool bad = s_bad != 0;
+    const bool ok = !bad && s_pre[B] <= top;
+    if (!ok && blockIdx.x == 0 && b == 0 && tid == 0)
+      set_status(t.status, bad ? 1 /* HSTU_ERR_INVALID_ARG */ : 2 /* HSTU_ERR_OUT_OF_PAGES */);
+    if (tid == 0) s_ok = ok;
+    u = s_u[b];
+    len = s_len[b];
+    held = s_held[b];
+    need = s_need[b];
+    pre = s_pre[b];
+  } else {
+    if (tid == 0) s_ok = *t.step_ok != 0;
+    u = users[b];
+    const bool known = u >= 0 && u < t.max_users;
+    len = known ? t.lengths[u] : 0;
+    held = known ? t.n_held[u] : 0;
+  }
+  __syncthreads();
+  const bool ok = s_ok != 0;
+  const bool known = u >= 0 && u < t.max_users;
+  const int32_t* list = t.page_lists + (known ? u : 0) * (int64_t)t.max_ppu;
+  const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
+  if (ok && tok0 < n) {
+    const int row_vec = t.H * t.d * ESZ / 16;  // 16-byte vectors per token row
+    const int vec_per_head = t.d * ESZ / 16;
+    const int ntok = (int)((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok);
+    const int64_t s0 = new_offsets[b];
+    for (int i = tid; i < ntok * row_vec * 2; i += kCopyThreads) {
+      const int kv = i / (ntok * row_vec);
+      const int rem = i % (ntok * row_vec);
+      const int tk = rem / row_vec, v = rem % row_vec;
+      const int h = v / vec_per_head, e16 = v % vec_per_head;
+      const int64_t pos = len + tok0 + tk;
+      const int64_t pi = pos / t.page_size;
+      // pages this step pops come straight from the stack (PLAN); the rest
+      // are on the user's list
+      const int32_t page = (PLAN && pi >= held) ? t.free_stack[top - 1 - (pre + (pi - held))]
+                                                : list[pi];
+      const int slot = (int)(pos % t.page_size);
+      const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + tk) * src_row_bytes;
+      const uint4 x = reinterpret_cast<const uint4*>(src)[v];
+      uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
+                     ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
+      reinterpret_cast<uint4*>(dst)[e16] = x;
+    }
+  }
+  if (blockIdx.x == 0) {
+    const int64_t flen = !known ? 0 : (ok ? len + n : len);
+    const int fheld = !known ? 0 : ((PLAN && ok) ? held + need : held);
+    if (PLAN && ok) {
+      int32_t* wlist = t.page_lists + u * (int64_t)t.max_ppu;
+      for (int k = tid; k < need; k += kCopyThreads) wlist[held + k] = t.free_stack[top - 1 - (pre + k)];
+    }
+    if (tid == 0 && cached_len_out) cached_len_out[b] = flen;
+    if (page_table_out) {
+      for (int p = tid; p < max_pages; p += kCopyThreads) {
+        int32_t pg = -1;
+        if (p < fheld) pg = (PLAN && p >= held) ? t.free_stack[top - 1 - (pre + (p - held))] : list[p];
+        page_table_out[(int64_t)b * max_pages + p] = pg;
+      }
+    }
+  }
+  if (!ok) return;  // the same verdict in every CTA (every thread of it)
+  __syncthreads();
+  if (PLAN) {
+    if (tid == 0) {
+      __threadfence();
+      const int prev = atomicAdd(t.step_done, 1);
+      s_last = prev == (int)(gridDim.x * gridDim.y) - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid < B) {
+      const int64_t ui = s_u[tid];
+      t.lengths[ui] = s_len[tid] + (new_offsets[tid + 1] - new_offsets[tid]);
+      t.n_held[ui] = s_held[tid] + s_need[tid];
+    }
+    if (tid == 0) {
+      *t.free_top = (int32_t)(top - s_pre[B]);
+      *t.step_done = 0;
+    }
+    __threadfence();
+  } else {
+    // the last CTA of this user commits the new length
+    const int n_chunks = (int)((n + kAppendTok - 1) / kAppendTok);
+    if (tid == 0 && tok0 < n) {
+      __threadfence();
+      const int prev = atomicAdd(&t.done[u], 1);
+      if (prev == n_chunks - 1) {
+        t.lengths[u] = len + n;
+        t.done[u] = 0;
+        __threadfence();
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order) {
@@ -341,6 +552,14 @@ cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order
   if (e != cudaSuccess) return e;
   e = cudaMemset(t->status, 0, sizeof(int32_t));
   if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->step_done, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->step_done, 0, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&t->step_ok, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(t->step_ok, 0, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
   std::vector<int32_t> order((size_t)t->n_pages);
   for (int64_t i = 0; i < t->n_pages; ++i) order[i] = host_free_order ? host_free_order[i] : (int32_t)i;
   if (t->n_pages > 0) {
@@ -364,6 +583,8 @@ void kv_table_free_storage(KvTableDev* t) {
   cudaFree(t->alloc_calls);
   cudaFree(t->done);
   cudaFree(t->status);
+  cudaFree(t->step_done);
+  cudaFree(t->step_ok);
 }
 
 cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int64_t* n_new, int B,
@@ -372,7 +593,8 @@ cudaError_t kv_alloc_launch(const KvTableDev& t, const int64_t* users, const int
   if (B == 0 && page_ids_out == nullptr) return cudaSuccess;
   if (n_new == nullptr && new_offsets == nullptr) return cudaErrorInvalidValue;
   return launch_dependent(kv_alloc_kernel, dim3(1), dim3(kAllocThreads), 0, stream, t, users, n_new,
-                          new_offsets, B, page_ids_out, page_ids_cap);
+                          new_offsets, B, page_ids_out, page_ids_cap, (int32_t*)nullptr,
+                          (int64_t)-1);
 }
 
 cudaError_t kv_release_launch(const KvTableDev& t, const int64_t* users, int B,
@@ -411,6 +633,41 @@ cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
   return launch_dependent(kv_lookup_kernel<4>, grid, dim3(kCopyThreads), 0, stream, t, users,
                           cached_len_out, page_table_out, max_pages, (uint8_t*)k_out,
                           (uint8_t*)v_out, out_offsets);
+}
+
+cudaError_t kv_step_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
+                           const void* v_new, const int64_t* new_offsets, int B, int max_new,
+                           int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
+                           cudaStream_t stream, int64_t src_row_elems) {
+  if (B == 0) return cudaSuccess;
+  if (B < 0 || B > 65535 || max_new < 0 || max_pages < 0) return cudaErrorInvalidValue;
+  const int64_t row_elems = src_row_elems > 0 ? src_row_elems : (int64_t)t.H * t.d;
+  if (row_elems < (int64_t)t.H * t.d || (row_elems * t.esize) % 16 != 0)
+    return cudaErrorInvalidValue;
+  if (page_table_out == nullptr) max_pages = 0;
+  const dim3 grid(std::max(1, (max_new + kAppendTok - 1) / kAppendTok), B);
+  const int64_t rb = row_elems * t.esize;
+  const uint8_t* k = (const uint8_t*)k_new;
+  const uint8_t* v = (const uint8_t*)v_new;
+  if (B <= kStepMaxUsers) {
+    if (t.esize == 2)
+      return launch_dependent(kv_step_kernel<2, true>, grid, dim3(kCopyThreads), 0, stream, t, users,
+                              k, v, new_offsets, B, max_new, rb, cached_len_out, page_table_out,
+                              max_pages);
+    return launch_dependent(kv_step_kernel<4, true>, grid, dim3(kCopyThreads), 0, stream, t, users, k,
+                            v, new_offsets, B, max_new, rb, cached_len_out, page_table_out,
+                            max_pages);
+  }
+  cudaError_t e = launch_dependent(kv_alloc_kernel, dim3(1), dim3(kAllocThreads), 0, stream, t, users,
+                                   (const int64_t*)nullptr, new_offsets, B, (int32_t*)nullptr, 0,
+                                   t.step_ok, (int64_t)max_new);
+  if (e != cudaSuccess) return e;
+  if (t.esize == 2)
+    return launch_dependent(kv_step_kernel<2, false>, grid, dim3(kCopyThreads), 0, stream, t, users, k,
+                            v, new_offsets, B, max_new, rb, cached_len_out, page_table_out,
+                            max_pages);
+  return launch_dependent(kv_step_kernel<4, false>, grid, dim3(kCopyThreads), 0, stream, t, users, k, v,
+                          new_offsets, B, max_new, rb, cached_len_out, page_table_out, max_pages);
 }
 
 }  // namespace hstu

@@ -22,6 +22,8 @@ struct KvTableDev {
   int32_t* alloc_calls;  // device counter of alloc launches (the next call's epoch - 1)
   int32_t* done;
   int32_t* status;
+  int32_t* step_done;  // CTAs of a fused step launch that finished (always back to 0)
+  int32_t* step_ok;    // the last alloc of a two-launch step succeeded (1) or not (0)
 };
 
 cudaError_t kv_table_alloc_storage(KvTableDev* t, const int32_t* host_free_order);
@@ -37,6 +39,12 @@ cudaError_t kv_release_launch(const KvTableDev& t, const int64_t* users, int B,
 cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
                              const void* v_new, const int64_t* new_offsets, int B, int max_new,
                              cudaStream_t stream, int64_t src_row_elems = 0);
+// One serving step: alloc (counts from new_offsets), append and lookup rows
+// (cached_len_out / page_table_out optional) as one all-or-nothing operation.
+cudaError_t kv_step_launch(const KvTableDev& t, const int64_t* users, const void* k_new,
+                           const void* v_new, const int64_t* new_offsets, int B, int max_new,
+                           int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
+                           cudaStream_t stream, int64_t src_row_elems = 0);
 cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
                              int64_t* cached_len_out, int32_t* page_table_out, int max_pages,
                              void* k_out, void* v_out, const int64_t* out_offsets, int max_len,

@@ -194,6 +194,31 @@ HSTU_API hstu_status hstu_kv_lookup(hstu_kv_table* t, const int64_t* users, int3
                            cudaStream_t stream);
 
 /*
+ * One serving step of the table ("NVIDIA Dynamo-Triton Gets End-to-End HSTU
+ * Generative Recommender Workflow", section "What the workflow combines":
+ * allocation, append and lookup of the paged KV data table): the effect of
+ * hstu_kv_alloc with n_new[b] = new_offsets[b+1] - new_offsets[b], then
+ * hstu_kv_append, then hstu_kv_lookup without the K/V gather, in one call.
+ *  users: int64 [B] device, unique, in [0, max_users).
+ *  k_new, v_new: [T_new, H, d] device, table dtype, 16-byte aligned (may be
+ *    NULL when max_new = 0); new_offsets: int64 [B+1] device.
+ *  max_new: bound on every user's new-token count (launch sizing); a larger
+ *    count is an invalid argument.
+ *  cached_len_out: int64 [B] (optional) = cached length after the step;
+ *  page_table_out: int32 [B, max_pages] (optional) = page lists, -1 padded.
+ * All or nothing: duplicate or out-of-range users, a negative or too large
+ * count (HSTU_ERR_INVALID_ARG) or too few free pages (HSTU_ERR_OUT_OF_PAGES)
+ * leave the table unchanged and record the status word; the lookup outputs
+ * then show the unchanged table.  Pages are popped exactly as hstu_kv_alloc
+ * pops them, so page ids match the three separate calls bit for bit.  Up to
+ * 64 users run as one kernel launch; larger batches as two.
+ */
+HSTU_API hstu_status hstu_kv_step(hstu_kv_table* t, const int64_t* users, const void* k_new,
+                                  const void* v_new, const int64_t* new_offsets, int32_t B,
+                                  int32_t max_new, int64_t* cached_len_out,
+                                  int32_t* page_table_out, int32_t max_pages, cudaStream_t stream);
+
+/*
  * Attention whose history K/V comes from the KV table, read page by page inside
  * the kernel (no gather).  users: int64 [B]; q_offsets: int64 [B+1] jagged
  * query rows; q: [Tq, H, d]; out: [Tq, H, d]; the table's dtype.
