@@ -228,10 +228,9 @@ class PagedPart:
         return float(pairs * c.H * 4 * c.d), bytes_, float(nq.sum())
 
     def kv_ops(self, stream=None):
-        t = self.table
-        t.alloc(self.users, self.n_new, stream=stream)
-        t.append(self.users, self.new_k, self.new_v, self.new_off, int(self.case.n_new.max()), stream=stream)
-        t.lookup(self.users, self.cached_len, self.page_table, stream=stream)
+        """alloc + append + lookup rows of this step's new tokens (one hstu_kv_step call)."""
+        self.table.step(self.users, self.new_k, self.new_v, self.new_off, int(self.case.n_new.max()),
+                        self.cached_len, self.page_table, stream=stream)
 
     def launch_attention(self, stream=None):
         h, c = self.hstu, self.case
@@ -520,6 +519,38 @@ def run_gpu(args):
 
     beam = {} if args.no_serving else BeamDecodePart().measure(flush_buf, hbm_peak, tf_peak)
 
+    # the cached-candidate step at larger batches (same per-user shapes): how far
+    # the fixed per-step latencies are amortised once a step moves more bytes
+    by_batch = {}
+    if not args.no_serving:
+        for nb in (32, 128):
+            part = PagedPart(W.cached_cand(B=nb, seed=2003 + 7919 * rank), 12, seed=91 + rank)
+            for _ in range(3):
+                part.kv_ops(); part.attention()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                part.kv_ops()
+                part.launch_attention()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            tot = byt = nq = 0.0
+            for _ in range(5):
+                flush_buf.fill_(1)
+                _, b_, q_ = part.units()
+                e0.record(); g.replay(); e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1) / 1e3
+                byt += b_
+                nq += q_
+                part.advance()
+            if part.table.status():
+                raise RuntimeError("KV table error in the batch-scaling measurement")
+            by_batch[f"B_{nb}"] = {"ms": round(tot / 5 * 1e3, 4),
+                                   "candidates_per_s": round(nq / tot, 1),
+                                   "hbm_gbs": round(byt / tot / 1e9, 1),
+                                   "frac_of_hbm": round(byt / tot / 1e9 / hbm_peak, 4)}
+            del g, part
+
     e2e = run_e2e(A, Bp, flush_buf, args) if rank == 0 else None
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
@@ -543,6 +574,7 @@ def run_gpu(args):
                 "cached_candidates": {"ms": round(t_b / args.steps * 1e3, 4),
                                       "candidates_per_s": round(cand_per_s, 1),
                                       "hbm_gbs": round(b_gbs, 1), "frac_of_hbm": round(b_gbs / hbm_peak, 4)},
+                "cached_candidates_by_batch": by_batch,
                 "cached_serving": serving,
                 "beam_decode": beam,
                 "jagged_bf16": {"ms": round(jt / jsteps * 1e3, 4),
