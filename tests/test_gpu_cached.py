@@ -238,6 +238,46 @@ def test_fp32_table_candidates_simt():
     t.close()
 
 
+def test_candidates_ragged_counts_many_users():
+    """37 users with different candidate counts (none, one, a tile, a tile and
+    a row, several tiles) and histories from empty to a few thousand tokens:
+    the key splits of every (head, query tile) are summed by whichever split
+    finishes last; a second call gives the same bits (every arrival counter
+    went back to zero)."""
+    import generative_recommender_sequence_b200 as hstu
+    rng = np.random.default_rng(31)
+    B, H, d = 37, 4, 128
+    hist = rng.integers(0, 3000, size=B)
+    hist[:3] = [0, 31, 2999]
+    n_cand = rng.choice([0, 1, 5, 128, 129, 200], size=B)
+    n_cand[0] = 7
+    n_new = 16
+    draw = lambda n: workloads._as_storage(rng.standard_normal((n, H, d), dtype=np.float32), "bf16")
+    need = int(np.sum((hist + n_new + 31) // 32))
+    n_pages = need + 9
+    case = workloads.CachedCase("ragged", H, d, hist.astype(np.int64), np.full(B, n_new, np.int64),
+                                draw(int(hist.sum())), draw(int(hist.sum())), draw(B * n_new),
+                                draw(B * n_new), rng.normal(0, 0.1, 16).astype(np.float32), n_pages,
+                                rng.permutation(n_pages).astype(np.int32), mode=0,
+                                n_cand=n_cand.astype(np.int64), q_cand=draw(int(n_cand.sum())),
+                                k_cand=draw(int(n_cand.sum())), v_cand=draw(int(n_cand.sum())),
+                                scale=1.0 / int((hist + n_new + n_cand).max()))
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), "ragged candidates", ulp_aware=True)
+    again = hstu.attn_cached_fwd(table, users, storage(case.q_cand, "bf16"), dev(case.q_offsets),
+                                 int(n_cand.max()), int(case.total_lengths.max()),
+                                 hstu.HSTU_MASK_CANDIDATES, k_cand=storage(case.k_cand, "bf16"),
+                                 v_cand=storage(case.v_cand, "bf16"), pos_table=dev(case.pos_table),
+                                 scale=case.scale)
+    torch.cuda.synchronize()
+    assert hstu.last_device_error() == 0
+    assert torch.equal(out, again)
+    table.close()
+
+
 def test_step_replayed_from_a_cuda_graph():
     """alloc + append + lookup + candidate attention captured once and replayed
     twice: each replay appends the delta again into fresh pages (the alloc epoch
