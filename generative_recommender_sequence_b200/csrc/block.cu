@@ -161,15 +161,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
       const int mt = t / n_tiles, nt = t % n_tiles;
       const uint32_t ab = tcount & 1;
+      const int64_t row = (int64_t)mt * GBM + r;
+      const bool valid = row < P.M;
+      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN;
+      // residual epilogue: this thread's whole row segment of X is loaded
+      // before the accumulator is ready (one memory latency per tile, hidden
+      // behind the main loop, instead of one per 32-column chunk)
+      uint4 res[EPI == EPI_RESIDUAL ? GBN / 8 : 1];
+      if (EPI == EPI_RESIDUAL && valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(orow);
+#pragma unroll
+        for (int q = 0; q < GBN / 8; ++q) res[q] = src[q];
+      }
       if (!mbar_wait_warp(smem_u32(&sm.acc_full[ab]), (tcount >> 1) & 1)) {
         if (lane == 0) atomicExch(P.err, DEV_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
-      const int64_t row = (int64_t)mt * GBM + r;
-      const bool valid = row < P.M;
-      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN;
-#pragma unroll 1
+#pragma unroll
       for (int ch = 0; ch < GBN / 32; ++ch) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_addr + ab * GBN + ch * 32, v);
@@ -190,10 +199,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             x[j] = fmaf(h, tanh_approx(h), h);
           }
         } else {
-          const uint4* res = reinterpret_cast<const uint4*>(orow + ch * 32);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint4 u = res[q];
+            const uint4 u = res[EPI == EPI_RESIDUAL ? ch * 4 + q : 0];
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
