@@ -351,7 +351,24 @@ __global__ void __launch_bounds__(kCopyThreads)
   pdl_wait();
   int64_t u, len, top = 0;
   int held, need = 0, pre = 0;
-  const int64_t n = new_offsets[b + 1] - new_offsets[b];
+  const int64_t s0 = new_offsets[b];
+  const int64_t n = new_offsets[b + 1] - s0;
+  // this thread's first source vector depends on nothing the plan computes:
+  // load it now so its latency overlaps the plan's dependent loads
+  const int row_vec = t.H * t.d * ESZ / 16;  // 16-byte vectors per token row
+  const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
+  // (a count above max_new makes the batch invalid: nothing is read for it,
+  // and the buffers may then be null)
+  const int ntok = (int)(tok0 < n && n <= max_new
+                             ? ((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok)
+                             : 0);
+  uint4 x0 = make_uint4(0u, 0u, 0u, 0u);
+  if (tid < ntok * row_vec * 2) {
+    const int kv = tid / (ntok * row_vec);
+    const int rem = tid % (ntok * row_vec);
+    const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + rem / row_vec) * src_row_bytes;
+    x0 = reinterpret_cast<const uint4*>(src)[rem % row_vec];
+  }
   if (PLAN) {
     if (tid == 0) {
       s_bad = 0;
@@ -434,12 +451,8 @@ __global__ void __launch_bounds__(kCopyThreads)
   const bool ok = s_ok != 0;
   const bool known = u >= 0 && u < t.max_users;
   const int32_t* list = t.page_lists + (known ? u : 0) * (int64_t)t.max_ppu;
-  const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
   if (ok && tok0 < n) {
-    const int row_vec = t.H * t.d * ESZ / 16;  // 16-byte vectors per token row
     const int vec_per_head = t.d * ESZ / 16;
-    const int ntok = (int)((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok);
-    const int64_t s0 = new_offsets[b];
     for (int i = tid; i < ntok * row_vec * 2; i += kCopyThreads) {
       const int kv = i / (ntok * row_vec);
       const int rem = i % (ntok * row_vec);
@@ -452,8 +465,11 @@ __global__ void __launch_bounds__(kCopyThreads)
       const int32_t page = (PLAN && pi >= held) ? t.free_stack[top - 1 - (pre + (pi - held))]
                                                 : list[pi];
       const int slot = (int)(pos % t.page_size);
-      const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + tk) * src_row_bytes;
-      const uint4 x = reinterpret_cast<const uint4*>(src)[v];
+      uint4 x = x0;
+      if (i != tid) {
+        const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + tk) * src_row_bytes;
+        x = reinterpret_cast<const uint4*>(src)[v];
+      }
       uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
                      ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
       reinterpret_cast<uint4*>(dst)[e16] = x;
