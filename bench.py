@@ -521,8 +521,9 @@ def run_gpu(args):
 
     # the cached-candidate step at larger batches (same per-user shapes): how far
     # the fixed per-step latencies are amortised once a step moves more bytes
+    # (single-GPU runs only: the 128-user case draws ~1.3 GB of host inputs)
     by_batch = {}
-    if not args.no_serving:
+    if not args.no_serving and world == 1:
         for nb in (32, 128):
             part = PagedPart(W.cached_cand(B=nb, seed=2003 + 7919 * rank), 12, seed=91 + rank)
             for _ in range(3):
