@@ -149,6 +149,7 @@ struct KParams {
   float* partial;
   int64_t total_q;
   int* err;
+  int part_v8;   // partial buffer 32-byte aligned: store whole 32-byte sectors
 };
 
 // ------------------------------------------------------------ scheduling
@@ -1036,13 +1037,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!row_ok) continue;
         if (P.partial) {
+          // whole 32-byte sectors when the buffer allows: the scattered
+          // per-row partial stores drain faster than as 16-byte pieces
           float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
                        it.h * HD + ocol;
+          if (P.part_v8) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            reinterpret_cast<float4*>(dst)[j / 4] =
-                make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
-                            __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+            for (int j = 0; j < 32; j += 8) st_global_v8(dst + j, oa + j);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              reinterpret_cast<float4*>(dst)[j / 4] =
+                  make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
+                              __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+          }
         } else {
           __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + ocol;
           const float sc2 = P.scale;
@@ -1230,13 +1238,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.o_empty));
       if (row_ok) {
         if (P.partial) {
+          // whole 32-byte sectors when the buffer allows: the scattered
+          // per-row partial stores drain faster than as 16-byte pieces
           float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
                        it.h * HD + cbase;
+          if (P.part_v8) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            reinterpret_cast<float4*>(dst)[j / 4] =
-                make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
-                            __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+            for (int j = 0; j < 32; j += 8) st_global_v8(dst + j, oa + j);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              reinterpret_cast<float4*>(dst)[j / 4] =
+                  make_float4(__uint_as_float(oa[j]), __uint_as_float(oa[j + 1]),
+                              __uint_as_float(oa[j + 2]), __uint_as_float(oa[j + 3]));
+          }
         } else {
           __nv_bfloat16* dst = P.out + row * P.out_stride + it.h * HD + cbase;
           const float sc2 = P.scale;
@@ -1495,6 +1510,7 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
     const size_t need = attn_sm100_workspace_bytes(p, num_sms);
     if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
     kp.partial = reinterpret_cast<float*>(workspace);
+    kp.part_v8 = (reinterpret_cast<uintptr_t>(workspace) & 31) == 0 ? 1 : 0;
   }
   // Paged causal attention over long query runs may go to CTA pairs: each pair
   // shares every K/V tile (each CTA loads half), halving the tile traffic into
