@@ -35,6 +35,10 @@ def test_host_argument_checks_need_no_gpu():
                                     ctypes.byref(out)) == 1
     assert lib.hstu_block_fwd(None, None, 1, 1, 1, 1, 512, 4, 64, None, None, None, 1.0, 1e-5,
                               None, 0, None) == 4
+    # the one-call KV step: no table, a negative batch or bound, missing offsets
+    assert lib.hstu_kv_step(None, None, None, None, None, 1, 1, None, None, 0, None) == 1
+    assert lib.hstu_kv_step(None, None, None, None, None, -1, 1, None, None, 0, None) == 1
+    assert lib.hstu_kv_step(None, None, None, None, None, 1, -1, None, None, 0, None) == 1
 
 
 def test_oracle_is_not_imported_by_the_product_package():
