@@ -552,7 +552,15 @@ def run_gpu(args):
                                    "frac_of_hbm": round(byt / tot / 1e9 / hbm_peak, 4)}
             del g, part
 
-    e2e = run_e2e(A, Bp, flush_buf, args) if rank == 0 else None
+    # every rank runs the end-to-end steps: whole-job units over the slowest rank
+    e2e_local = run_e2e(A, Bp, flush_buf, args)
+    e2e_t = max_over_ranks(e2e_local.pop("seconds"), world)
+    e2e_units = sum_over_ranks(e2e_local.pop("flops"), world)
+    e2e_h2d = sum_over_ranks(float(e2e_local["h2d_bytes_per_step"]), world)
+    e2e_d2h = sum_over_ranks(float(e2e_local["d2h_bytes_per_step"]), world)
+    e2e = {"value": round(e2e_units / e2e_t / 1e12, 4), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(e2e_h2d), "d2h_bytes_per_step": int(e2e_d2h),
+           "steps": e2e_local["steps"]}
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
         c5 = A.case
@@ -601,7 +609,9 @@ def run_gpu(args):
 
 def run_e2e(A, Bp, flush_buf, args):
     """Same metric through the public API with host (pinned) inputs: H2D of each
-    step's inputs and D2H of its outputs are inside the timed region."""
+    step's inputs and D2H of its outputs are inside the timed region.  Returns
+    this rank's device seconds, FLOPs and bytes per step (the caller reduces
+    them over ranks)."""
     import torch
     parts = [(A, ["q", "new_k", "new_v"]), (Bp, ["q", "k_c", "v_c", "new_k", "new_v"])]
     host, saved = [], []
@@ -635,7 +645,7 @@ def run_e2e(A, Bp, flush_buf, args):
         flops += fa + fb
     for part, n, t in saved:
         setattr(part, n, t)
-    return {"value": round(flops / tot / 1e12, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+    return {"seconds": tot, "flops": flops, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps}
 
 
