@@ -70,6 +70,12 @@ def last_device_error(stream=None) -> int:
     return load().hstu_last_device_error(_stream(stream))
 
 
+def wait_timeout_selftest(timeout_us: int = 20000, stream=None) -> None:
+    """Run the bounded-wait self test: a GPU wait that nothing completes gives up
+    after timeout_us and records HSTU_ERR_TIMEOUT for last_device_error()."""
+    check("hstu_wait_timeout_selftest", load().hstu_wait_timeout_selftest(int(timeout_us), _stream(stream)))
+
+
 def attn_fwd(q, k, v, seq_offsets, max_len: int, pos_table=None, time_table=None, timestamps=None,
              scale: float = 1.0, out=None, stream=None) -> torch.Tensor:
     """Jagged causal HSTU attention; q, k, v: [T, H, d] (bf16 or fp32), seq_offsets int64 [B+1]."""

@@ -62,6 +62,7 @@ _SIGNATURES = {
     "hstu_user_map_status": ([_P, _P], _I32),
     "hstu_kv_lookup": ([_P, _P, _I32, _P, _P, _I32, _P, _P, _P, _I32, _P], _I32),
     "hstu_kv_step": ([_P, _P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _P], _I32),
+    "hstu_wait_timeout_selftest": ([_I32, _P], _I32),
     "hstu_attn_cached_fwd": ([_P, _P, _I32, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _F, _P, _P,
                               _SZ, _P], _I32),
     "hstu_attn_cached_workspace_size": ([_P, _I32, _I64, _I32, _I32, _I32], _SZ),

@@ -16,6 +16,7 @@
 #include "beam_decode.h"
 #include "block.h"
 #include "kv_table.h"
+#include "selftest.h"
 #include "user_map.h"
 
 // Device error word written by kernels whose bounded waits ran out.
@@ -179,6 +180,11 @@ hstu_status hstu_last_device_error(cudaStream_t stream) {
     cudaMemcpyToSymbol(g_hstu_device_error, &z, sizeof(int));
   }
   return (hstu_status)v;
+}
+
+hstu_status hstu_wait_timeout_selftest(int32_t timeout_us, cudaStream_t stream) {
+  if (timeout_us < 1 || timeout_us > 2000000) return HSTU_ERR_INVALID_ARG;
+  return from_cuda(wait_timeout_selftest_launch(device_error_word(), (int64_t)timeout_us * 1000, stream));
 }
 
 hstu_status hstu_attn_fwd(const void* q, const void* k, const void* v, const int64_t* seq_offsets,

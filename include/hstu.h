@@ -94,6 +94,14 @@ HSTU_API const char* hstu_status_string(hstu_status s);
  * then undefined), HSTU_OK otherwise. */
 HSTU_API hstu_status hstu_last_device_error(cudaStream_t stream);
 
+/* Failure-detection self test: one GPU thread waits, for at most timeout_us
+ * microseconds (1 .. 2 000 000), on an mbarrier that nothing completes, then
+ * records HSTU_ERR_TIMEOUT in the device error word that hstu_last_device_error
+ * reads -- the bounded wait and error path of every kernel in the library.  No
+ * fault, trap or unbounded wait is involved and the context stays usable.
+ * Returns HSTU_ERR_INVALID_ARG for a limit outside that range. */
+HSTU_API hstu_status hstu_wait_timeout_selftest(int32_t timeout_us, cudaStream_t stream);
+
 /*
  * Jagged causal HSTU attention (section "HSTU" of the page cited above): user
  * b owns tokens [seq_offsets[b], seq_offsets[b+1]); token i attends to the

@@ -35,6 +35,9 @@ def test_host_argument_checks_need_no_gpu():
                                     ctypes.byref(out)) == 1
     assert lib.hstu_block_fwd(None, None, 1, 1, 1, 1, 512, 4, 64, None, None, None, 1.0, 1e-5,
                               None, 0, None) == 4
+    # the bounded-wait self test refuses limits outside 1 us .. 2 s before any launch
+    assert lib.hstu_wait_timeout_selftest(0, None) == 1
+    assert lib.hstu_wait_timeout_selftest(2000001, None) == 1
     # the one-call KV step: no table, a negative batch or bound, missing offsets
     assert lib.hstu_kv_step(None, None, None, None, None, 1, 1, None, None, 0, None) == 1
     assert lib.hstu_kv_step(None, None, None, None, None, -1, 1, None, None, 0, None) == 1
