@@ -68,7 +68,7 @@ def _load():
             lib.oracle_attn_candidates.restype = I
             lib.oracle_layernorm_gate.argtypes = [L, L, P, P, D, I, P, I]
             lib.oracle_layernorm_gate.restype = I
-            lib.oracle_hstu_block.argtypes = [L, I, P, I, I, I, I, P, P, P, P, P, I, P, I, D, D, I, P, I]
+            lib.oracle_hstu_block.argtypes = [L, I, P, I, I, I, I, P, P, P, P, P, I, P, I, D, D, I, I, P, I]
             lib.oracle_hstu_block.restype = I
             _lib = lib
     return _lib
@@ -165,8 +165,12 @@ def layernorm_gate(a, u, eps=1e-5, round_bf16=False, threads=None) -> np.ndarray
 
 
 def hstu_block(x0, seq_offsets, w_uvqk, w_o, timestamps, pos_table, time_table, scale,
-               ln_eps=1e-5, H=4, dh=128, round_bf16=True, return_layers=False, threads=None):
-    """Block stack: per layer X <- X + (LayerNorm(attn(SiLU(X W1))) * U) W2."""
+               ln_eps=1e-5, H=4, dh=128, round_bf16=True, return_layers=False, threads=None,
+               round_output=True):
+    """Block stack: per layer X <- X + (LayerNorm(attn(SiLU(X W1))) * U) W2.
+
+    round_bf16 rounds UVQK, A, G and X to bf16 where the GPU stores bf16;
+    round_output=False leaves only the last layer's X unrounded."""
     x = _f64(x0).copy()
     off = _i64(seq_offsets)
     w1, w2 = _f64(w_uvqk), _f64(w_o)
@@ -178,7 +182,7 @@ def hstu_block(x0, seq_offsets, w_uvqk, w_o, timestamps, pos_table, time_table, 
     rc = _load().oracle_hstu_block(T, len(off) - 1, _p(off), n_layers, dm, H, dh, _p(x), _p(w1),
                                    _p(w2), _p(ts), _p(pt), 0 if pt is None else len(pt), _p(tt),
                                    0 if tt is None else len(tt), float(scale), float(ln_eps),
-                                   int(bool(round_bf16)), _p(layers),
+                                   int(bool(round_bf16)), int(bool(round_output)), _p(layers),
                                    threads or default_threads())
     if rc != 0:
         raise ValueError("oracle_hstu_block failed (%d)" % rc)

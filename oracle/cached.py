@@ -26,11 +26,13 @@ from . import hstu_block
 
 
 def hstu_block_cached(x_hist, hist_offsets, x_new, new_offsets, x_cand, cand_offsets, w_uvqk, w_o,
-                      pos_table, scale, ln_eps=1e-5, H=4, dh=128, round_bf16=True, threads=None):
+                      pos_table, scale, ln_eps=1e-5, H=4, dh=128, round_bf16=True, threads=None,
+                      round_output=True):
     """Returns (final new rows [T_new, d], final candidate rows [T_cand, d]) in fp64.
 
     x_hist / x_new / x_cand: layer-0 rows, jagged per user by the [B+1] offsets
-    (x_cand / cand_offsets may be None)."""
+    (x_cand / cand_offsets may be None).  round_output=False leaves the last
+    layer's output unrounded (see ``oracle.hstu_block``)."""
     ho, no = np.asarray(hist_offsets, np.int64), np.asarray(new_offsets, np.int64)
     B = len(ho) - 1
     co = np.zeros(B + 1, np.int64) if cand_offsets is None else np.asarray(cand_offsets, np.int64)
@@ -52,5 +54,5 @@ def hstu_block_cached(x_hist, hist_offsets, x_new, new_offsets, x_cand, cand_off
     offsets = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
     x_all = np.concatenate(seqs) if seqs else np.zeros((0, xh.shape[1]))
     y = hstu_block(x_all, offsets, w_uvqk, w_o, None, pos_table, None, scale, ln_eps=ln_eps, H=H,
-                   dh=dh, round_bf16=round_bf16, threads=threads)
+                   dh=dh, round_bf16=round_bf16, threads=threads, round_output=round_output)
     return y[np.asarray(new_rows, np.int64)], y[np.asarray(cand_rows, np.int64)]

@@ -338,14 +338,16 @@ int oracle_layernorm_gate(int64_t T, int64_t F, const double* a, const double* u
  * One layer: UVQK = SiLU(X W1); A = causal attention(Q, K, V) with the rab;
  *            G = LayerNorm(A) * U; X <- X + G W2.
  * With round_bf16 != 0 each materialised tensor (UVQK, A, G, X) is rounded to
- * bf16 (RNE), exactly where the GPU path stores bf16.
+ * bf16 (RNE), exactly where the GPU path stores bf16.  round_output == 0 keeps
+ * the last layer's X + G W2 unrounded (every other rounding point stays), so a
+ * caller can compare a bf16 result against the value before its final rounding.
  * layer_out: optional [n_layers, T, dm], X after every layer.
  */
 int oracle_hstu_block(int64_t T, int B, const int64_t* seq_offsets, int n_layers, int dm, int H,
                       int dh, double* x, const double* w_uvqk, const double* w_o,
                       const int64_t* timestamps, const double* pos_table, int n_pos,
                       const double* time_table, int n_time, double scale, double ln_eps,
-                      int round_bf16, double* layer_out, int n_threads) {
+                      int round_bf16, int round_output, double* layer_out, int n_threads) {
     if (T != seq_offsets[B]) return -1;
     int64_t F = (int64_t)H * dh, N1 = 4 * F;
     double* uvqk = (double*)malloc(sizeof(double) * T * N1);
@@ -370,9 +372,10 @@ int oracle_hstu_block(int64_t T, int B, const int64_t* seq_offsets, int n_layers
         run_tasks(lngate_task, &lc, T, n_threads);
         gemm_ctx g2 = {g, w_o + (int64_t)l * F * dm, d, F, dm, 0, 0};
         run_tasks(gemm_task, &g2, T, n_threads);
+        const int round_x = round_bf16 && (round_output || l + 1 < n_layers);
         for (int64_t i = 0; i < T * dm; i++) {
             double y = x[i] + d[i];
-            x[i] = round_bf16 ? oracle_round_bf16(y) : y;
+            x[i] = round_x ? oracle_round_bf16(y) : y;
         }
         if (layer_out) memcpy(layer_out + (int64_t)l * T * dm, x, sizeof(double) * T * dm);
     }
