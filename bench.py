@@ -13,12 +13,19 @@ two configurations the metric is quoted on:
      history L ~ U[1024, 4096] (100% KV hit); per step KV alloc + append of 64
      tokens per user, lookup, then 128 candidates per user attend to the whole
      cached history plus themselves ("cached candidates/sec").
-Every step appends into fresh pages (the pools are sized for all steps), so the
-histories grow; FLOPs and bytes are counted from the actual lengths of every
-step.  value = attention FLOPs of both parts (unmasked pairs only) / step time,
-in TFLOP/s.  The 8-user jagged workload (``jagged_bf16``) is timed separately
-and reported under parts.  Inputs are resident in HBM; L2 is flushed (256 MiB
-write) between steps, outside the per-step CUDA events.
+Before every step (outside the timed region) both tables are put back to the
+state after their prefill: the users are released and their histories
+allocated and appended again, so every timed step sees exactly the workloads'
+cached lengths (history + this step's append).  value = attention FLOPs of both
+parts (unmasked pairs only) / step time, in TFLOP/s.  The 8-user jagged workload
+(``jagged_bf16``), the 8-layer block stack (``block_stack``) and the KV append
+path are timed separately and reported under parts.  Inputs are resident in
+HBM; L2 is flushed (256 MiB write) between steps, outside the per-step CUDA
+events.
+
+``--gpus N`` without an outer launcher re-executes this script under
+torch.distributed.run with N local ranks (one process per GPU); under a
+launcher, WORLD_SIZE must equal N.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference this build
 has) on a bounded sample of the same workloads.
@@ -134,11 +141,25 @@ class ClockSampler:
         return out
 
 
+def launcher_command(n_gpus, argv, port=None):
+    """The torch.distributed.run command that starts one rank per GPU of this node."""
+    port = port if port is not None else 29500 + (os.getpid() % 2000)
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n_gpus}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def check_world(n_gpus, env):
+    """Rank layout from the launcher's environment; refuses a --gpus / WORLD_SIZE mismatch."""
+    world = int(env.get("WORLD_SIZE", "1"))
+    if "WORLD_SIZE" in env and world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but the launcher started WORLD_SIZE={world} ranks")
+    return int(env.get("RANK", "0")), world, int(env.get("LOCAL_RANK", "0"))
+
+
 def dist_setup(n_gpus):
     import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = check_world(n_gpus, os.environ)
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -172,27 +193,30 @@ def _dev(a, dt=None):
 
 
 class PagedPart:
-    """A cached workload (long_history or cached_cand) with a KV table sized for all steps."""
+    """A cached workload (long_history or cached_cand) in its own KV table.
 
-    def __init__(self, case, n_steps_total, seed):
+    reset() puts the table back to the state after the prefill (release every
+    user, then allocate and append the history again), so each step appends
+    the workload's new tokens onto exactly the workload's history."""
+
+    def __init__(self, case, seed):
         import torch
         import generative_recommender_sequence_b200 as hstu
         import workloads as W
         self.hstu, self.case = hstu, case
-        per_step_pages = int(np.max((case.n_new + 31) // 32)) + 1
-        extra = case.B * n_steps_total * per_step_pages
+        # room for the history + one step's append, plus a spare page per user
+        n_pages = max(case.n_pages, int(np.sum((case.total_lengths + 31) // 32)) + case.B)
         rng = np.random.default_rng(seed)
-        order = np.concatenate([case.free_order, case.n_pages + rng.permutation(extra)]).astype(np.int32)
-        self.max_cached = int(case.total_lengths.max()) + n_steps_total * int(case.n_new.max())
+        order = rng.permutation(n_pages).astype(np.int32)
+        self.max_cached = int(case.total_lengths.max())
         self.max_ppu = (self.max_cached + 31) // 32 + 2
-        self.table = hstu.KVTable(case.n_pages + extra, case.H, case.d, max_users=case.B,
+        self.table = hstu.KVTable(n_pages, case.H, case.d, max_users=case.B,
                                   max_pages_per_user=self.max_ppu, free_order=order)
         self.users = _dev(case.users)
-        hist_off = W.offsets_from_lengths(case.hist_lengths)
-        self.table.alloc(self.users, _dev(case.hist_lengths))
-        if int(case.hist_lengths.max()) > 0:
-            self.table.append(self.users, _dev(case.hist_k, "bf16"), _dev(case.hist_v, "bf16"),
-                              _dev(hist_off), int(case.hist_lengths.max()))
+        self.hist_len = _dev(case.hist_lengths)
+        self.hist_off = _dev(W.offsets_from_lengths(case.hist_lengths))
+        self.hist_k, self.hist_v = _dev(case.hist_k, "bf16"), _dev(case.hist_v, "bf16")
+        self.reset()
         assert self.table.status() == 0
         self.n_new = _dev(case.n_new)
         self.new_off = _dev(W.offsets_from_lengths(case.n_new))
@@ -208,15 +232,23 @@ class PagedPart:
         self.out = torch.empty_like(self.q)
         self.cached_len = torch.empty(case.B, dtype=torch.int64, device="cuda")
         self.page_table = torch.empty((case.B, self.max_ppu), dtype=torch.int32, device="cuda")
-        self.hist_now = case.hist_lengths.copy()
         need = self.table.workspace_size(case.B, int(case.q_offsets[-1]), int(self.n_q.max()),
                                          self.max_cached, case.mode)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
 
-    def units(self):
-        """(attention flops, algorithmic bytes, queries) of the next step."""
+    def reset(self, stream=None):
+        """Back to the prefilled state: release every user, re-append its history."""
         c = self.case
-        Lk = (self.hist_now + c.n_new).astype(np.float64)
+        self.table.release(self.users, stream=stream)
+        self.table.alloc(self.users, self.hist_len, stream=stream)
+        if int(c.hist_lengths.max()) > 0:
+            self.table.append(self.users, self.hist_k, self.hist_v, self.hist_off,
+                              int(c.hist_lengths.max()), stream=stream)
+
+    def units(self):
+        """(attention flops, algorithmic bytes, queries) of one step."""
+        c = self.case
+        Lk = (c.hist_lengths + c.n_new).astype(np.float64)
         nq = self.n_q.astype(np.float64)
         if c.mode == 0:
             pairs = (nq * (Lk + 1)).sum()
@@ -238,13 +270,8 @@ class PagedPart:
                           c.mode, k_cand=self.k_c, v_cand=self.v_c, pos_table=self.pt, scale=c.scale,
                           out=self.out, workspace=self.ws, stream=stream)
 
-    def advance(self):
-        """Host-side record of the cached lengths after one more step."""
-        self.hist_now = self.hist_now + self.case.n_new
-
     def attention(self, stream=None):
         self.launch_attention(stream)
-        self.advance()
 
 
 class JaggedPart:
@@ -424,19 +451,146 @@ class BeamDecodePart:
         return res
 
 
+class BlockStackPart:
+    """The 8-layer HSTU block stack of workload ``block_stack`` (B=8, L~U[512,4096],
+    d_model 512, 4 heads x 128, bf16, position + time rab): one hstu_block_fwd
+    call over all layers, replayed from a CUDA graph after an L2 flush.  The
+    attention alone (the same lengths and rab on contiguous Q/K/V) and one layer
+    are timed too, so GEMMs + LayerNorm gate = layer - attention."""
+
+    def __init__(self):
+        import torch
+        import generative_recommender_sequence_b200 as hstu
+        import workloads as W
+        self.hstu = hstu
+        c = W.block_stack()
+        self.c = c
+        self.x0 = _dev(c.x0, "bf16")
+        self.x = self.x0.clone()
+        self.off = _dev(c.seq_offsets)
+        self.w1 = [_dev(c.w_uvqk[l], "bf16") for l in range(c.n_layers)]
+        self.w2 = [_dev(c.w_o[l], "bf16") for l in range(c.n_layers)]
+        self.pt, self.tt, self.ts = _dev(c.pos_table), _dev(c.time_table), _dev(c.timestamps)
+        self.ws = torch.empty(hstu.block_workspace_size(c.T, c.d_model, c.H, c.dh),
+                              dtype=torch.uint8, device="cuda")
+        rng = np.random.default_rng(4)
+        qkv = lambda: _dev(W._as_storage(rng.standard_normal((c.T, c.H, c.dh), dtype=np.float32),
+                                         "bf16"), "bf16")
+        self.q, self.k, self.v = qkv(), qkv(), qkv()
+        self.a_out = torch.empty_like(self.q)
+
+    def stack(self, n_layers):
+        self.hstu.block_fwd(self.x, self.off, int(self.c.lengths.max()), self.w1[:n_layers],
+                            self.w2[:n_layers], pos_table=self.pt, time_table=self.tt,
+                            timestamps=self.ts, scale=self.c.scale, workspace=self.ws)
+
+    def attention(self):
+        self.hstu.attn_fwd(self.q, self.k, self.v, self.off, int(self.c.lengths.max()),
+                           pos_table=self.pt, time_table=self.tt, timestamps=self.ts,
+                           scale=self.c.scale, out=self.a_out)
+
+    def measure(self, flush_buf, tf_peak, reps=5):
+        import torch
+        c = self.c
+        res = {}
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        T = float(c.T)
+        gemm = 2 * T * c.d_model * (4 * c.H * c.dh) + 2 * T * (c.H * c.dh) * c.d_model
+        L = c.lengths.astype(np.float64)
+        attn = float((L * (L + 1) / 2).sum() * c.H * 4 * c.dh)
+        for name, fn, flops in (("stack", lambda: self.stack(c.n_layers), c.flops()),
+                                ("one_layer", lambda: self.stack(1), gemm + attn),
+                                ("attention", self.attention, attn)):
+            fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            tot = 0.0
+            for _ in range(reps):
+                self.x.copy_(self.x0)
+                flush_buf.fill_(1)
+                e0.record(); g.replay(); e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1) / 1e3
+            t = tot / reps
+            res[name + "_ms"] = round(t * 1e3, 4)
+            res[name + "_tflops"] = round(flops / t / 1e12, 2)
+            del g
+        res["gemm_ln_per_layer_ms"] = round(res["one_layer_ms"] - res["attention_ms"], 4)
+        res["frac_of_bf16_peak"] = round(res["stack_tflops"] / tf_peak, 4)
+        res["tokens"] = int(c.T)
+        if self.hstu.last_device_error():
+            raise RuntimeError("device error in the block stack measurement")
+        return res
+
+
+def kv_append_measure(A, Bp, flush_buf, hbm_peak, reps=5):
+    """The KV append path: (1) the serving steps' hstu_kv_step (alloc + append +
+    lookup rows: 8 users x 64 tokens, 32 users x 16 tokens), (2) a bulk append
+    of every long-history user's whole history into fresh pages (prefill /
+    onboarding).  Algorithmic bytes: each appended token's K and V read once
+    and written once (2 x H x d x 2 bytes each way)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    res = {}
+    for name, part in (("step_cached_cand", Bp), ("step_long_history", A)):
+        c = part.case
+        tok = float(c.n_new.sum())
+        byt = tok * c.H * c.d * 2 * 2 * 2
+        tot = 0.0
+        for _ in range(reps):
+            part.reset()
+            flush_buf.fill_(1)
+            e0.record(); part.kv_ops(); e1.record()
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1) / 1e3
+        t = tot / reps
+        res[name] = {"tokens": int(tok), "us": round(t * 1e6, 2), "gbs": round(byt / t / 1e9, 1),
+                     "frac_of_hbm": round(byt / t / 1e9 / hbm_peak, 4)}
+    c = A.case
+    tok = float(c.hist_lengths.sum())
+    byt = tok * c.H * c.d * 2 * 2 * 2
+    tot = 0.0
+    for _ in range(reps):
+        A.table.release(A.users)
+        A.table.alloc(A.users, A.hist_len)
+        flush_buf.fill_(1)
+        e0.record()
+        A.table.append(A.users, A.hist_k, A.hist_v, A.hist_off, int(c.hist_lengths.max()))
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1) / 1e3
+    t = tot / reps
+    res["bulk_append_long_history"] = {"tokens": int(tok), "us": round(t * 1e6, 2),
+                                       "gbs": round(byt / t / 1e9, 1),
+                                       "frac_of_hbm": round(byt / t / 1e9 / hbm_peak, 4)}
+    A.reset()
+    torch.cuda.synchronize()
+    if A.table.status() or Bp.table.status():
+        raise RuntimeError("KV table error in the append measurement")
+    return res
+
+
+def rank_seeds(rank):
+    """Weak scaling: every rank owns one per-GPU batch of distinct users, drawn
+    from its own seeds (rank 0 draws the reference workloads)."""
+    return {"long_history": 1005 + 7919 * rank, "cached_cand": 1003 + 7919 * rank,
+            "pool_long": 55 + rank, "pool_cand": 77 + rank}
+
+
 def run_gpu(args):
     import torch
     import workloads as W
     rank, world, local = dist_setup(args.gpus)
     hbm_peak, tf_peak, tf_sus, peak_src = load_peaks()
-    n_total = args.warmup + args.steps + 12
-    # weak scaling: every rank owns one per-GPU batch of distinct users (its own
-    # seeds; rank 0 draws the reference workloads), no data-path collective
-    A = PagedPart(W.long_history(seed=1005 + 7919 * rank), n_total, seed=55 + rank)
-    Bp = PagedPart(W.cached_cand(seed=1003 + 7919 * rank), n_total, seed=77 + rank)
+    seeds = rank_seeds(rank)
+    A = PagedPart(W.long_history(seed=seeds["long_history"]), seed=seeds["pool_long"])
+    Bp = PagedPart(W.cached_cand(seed=seeds["cached_cand"]), seed=seeds["pool_cand"])
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
     for _ in range(args.warmup):
+        A.reset(); Bp.reset()
         flush_buf.fill_(1)
         A.kv_ops(); A.attention(); Bp.kv_ops(); Bp.attention()
     torch.cuda.synchronize()
@@ -444,8 +598,8 @@ def run_gpu(args):
         raise RuntimeError("device error during warm-up")
 
     # The step's launches as CUDA graphs (capture does not execute them): the KV
-    # ops read and advance the table state on the device, so every replay
-    # appends into fresh slots exactly like a direct call.
+    # step reads the table state on the device, so every replay after a reset
+    # appends onto exactly the prefilled history.
     g_akv, g_aat, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_akv):
         A.kv_ops()
@@ -455,9 +609,17 @@ def run_gpu(args):
         Bp.kv_ops()
         Bp.launch_attention()
     torch.cuda.synchronize()
+    # kernels of this library per step: long history KV step + attention; cached
+    # candidates KV step + attention + split reduce (when its keys are split)
+    # (a split leaves partial sums in the workspace, so a non-zero workspace
+    # size means the reduce kernel runs)
+    split = lambda P: P.table.workspace_size(P.case.B, int(P.case.q_offsets[-1]), int(P.n_q.max()),
+                                             P.max_cached, P.case.mode) > 0
+    launches_per_step = 2 + int(split(A)) + 2 + int(split(Bp))
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    fa = fb = bb = qb = 0.0
+    fa, _, _ = A.units()
+    fb, bb, qb = Bp.units()
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -466,9 +628,8 @@ def run_gpu(args):
         time.sleep(0.25)
     wall0 = time.perf_counter()
     for i in range(args.steps):
+        A.reset(); Bp.reset()
         flush_buf.fill_(1)
-        f_a, _, _ = A.units()
-        f_b, b_b, q_b = Bp.units()
         ev[i][0].record()
         g_akv.replay()
         ev[i][1].record()
@@ -476,9 +637,6 @@ def run_gpu(args):
         ev[i][2].record()
         g_b.replay()
         ev[i][3].record()
-        A.advance()
-        Bp.advance()
-        fa += f_a; fb += f_b; bb += b_b; qb += q_b
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - wall0
@@ -490,24 +648,47 @@ def run_gpu(args):
     if A.table.status() or Bp.table.status() or A.hstu.last_device_error():
         raise RuntimeError("device error during the timed steps")
     t_max = max_over_ranks(t_step, world)
-    value = sum_over_ranks(fa + fb, world) / t_max / 1e12
-    a_tflops = fa / (t_akv + t_aat) / 1e12
-    a_attn_tflops = fa / t_aat / 1e12
-    cand_per_s = qb / t_b
-    b_gbs = bb / t_b / 1e9
+    value = sum_over_ranks((fa + fb) * args.steps, world) / t_max / 1e12
+    a_tflops = fa * args.steps / (t_akv + t_aat) / 1e12
+    a_attn_tflops = fa * args.steps / t_aat / 1e12
+    cand_per_s = qb * args.steps / t_b
+    b_gbs = bb * args.steps / t_b / 1e9
+
+    # the candidate kernels alone (attention + split reduce, no KV step): the
+    # bytes they must move are the cached K/V (history + append) and the
+    # candidates' Q, K, V in and O out
+    g_bat = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_bat):
+        Bp.launch_attention()
+    t_bat = 0.0
+    nb_at = max(5, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c3 = Bp.case
+    Lk3 = (c3.hist_lengths + c3.n_new).astype(np.float64)
+    row3 = c3.H * c3.d * 2
+    b_at = float((Lk3 * 2 * row3).sum() + c3.n_cand.sum() * row3 * 4)
+    for _ in range(nb_at):
+        flush_buf.fill_(1)
+        e0.record(); g_bat.replay(); e1.record()
+        torch.cuda.synchronize()
+        t_bat += e0.elapsed_time(e1) / 1e3
+    t_bat /= nb_at
+    del g_bat
 
     # the jagged workload, reported beside the step (not part of value)
     J = JaggedPart()
     for _ in range(3):
         J.run()
     jt = 0.0
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(max(3, args.steps // 2)):
+    jsteps = max(3, args.steps // 2)
+    for _ in range(jsteps):
         flush_buf.fill_(1)
         e0.record(); J.run(); e1.record()
         torch.cuda.synchronize()
         jt += e0.elapsed_time(e1) / 1e3
-    jsteps = max(3, args.steps // 2)
+
+    block = {} if args.no_serving else BlockStackPart().measure(flush_buf, tf_peak)
+    kv_append = kv_append_measure(A, Bp, flush_buf, hbm_peak)
 
     # KV-cached multi-layer serving vs the uncached stack, reported beside the step
     serving = {}
@@ -525,31 +706,28 @@ def run_gpu(args):
     by_batch = {}
     if not args.no_serving and world == 1:
         for nb in (32, 128):
-            part = PagedPart(W.cached_cand(B=nb, seed=2003 + 7919 * rank), 12, seed=91 + rank)
+            part = PagedPart(W.cached_cand(B=nb, seed=2003 + 7919 * rank), seed=91 + rank)
             for _ in range(3):
-                part.kv_ops(); part.attention()
+                part.reset(); part.kv_ops(); part.attention()
             torch.cuda.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 part.kv_ops()
                 part.launch_attention()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            tot = byt = nq = 0.0
+            tot = 0.0
+            _, b_, q_ = part.units()
             for _ in range(5):
+                part.reset()
                 flush_buf.fill_(1)
-                _, b_, q_ = part.units()
                 e0.record(); g.replay(); e1.record()
                 torch.cuda.synchronize()
                 tot += e0.elapsed_time(e1) / 1e3
-                byt += b_
-                nq += q_
-                part.advance()
             if part.table.status():
                 raise RuntimeError("KV table error in the batch-scaling measurement")
             by_batch[f"B_{nb}"] = {"ms": round(tot / 5 * 1e3, 4),
-                                   "candidates_per_s": round(nq / tot, 1),
-                                   "hbm_gbs": round(byt / tot / 1e9, 1),
-                                   "frac_of_hbm": round(byt / tot / 1e9 / hbm_peak, 4)}
+                                   "candidates_per_s": round(q_ * 5 / tot, 1),
+                                   "hbm_gbs": round(b_ * 5 / tot / 1e9, 1),
+                                   "frac_of_hbm": round(b_ * 5 / tot / 1e9 / hbm_peak, 4)}
             del g, part
 
     # every rank runs the end-to-end steps: whole-job units over the slowest rank
@@ -573,7 +751,8 @@ def run_gpu(args):
                        "seq_len": int(c5.total_lengths.max()),
                        "parallelism": f"dp{world} (users sharded, no collective on the data path)",
                        "l2": "flushed between steps (256 MiB write, outside the step events)",
-                       "timing": "CUDA-graph replay of each part, CUDA events between replays"},
+                       "timing": "tables reset to the prefilled state before every step (outside "
+                                 "the events); CUDA-graph replay of each part, CUDA events between replays"},
             "parts": {
                 "long_history": {"ms": round((t_akv + t_aat) / args.steps * 1e3, 4),
                                  "kv_ops_ms": round(t_akv / args.steps * 1e3, 4),
@@ -582,8 +761,13 @@ def run_gpu(args):
                                  "frac_of_bf16_peak": round(a_attn_tflops / tf_peak, 4)},
                 "cached_candidates": {"ms": round(t_b / args.steps * 1e3, 4),
                                       "candidates_per_s": round(cand_per_s, 1),
-                                      "hbm_gbs": round(b_gbs, 1), "frac_of_hbm": round(b_gbs / hbm_peak, 4)},
+                                      "hbm_gbs": round(b_gbs, 1), "frac_of_hbm": round(b_gbs / hbm_peak, 4),
+                                      "attention_only_us": round(t_bat * 1e6, 2),
+                                      "attention_only_gbs": round(b_at / t_bat / 1e9, 1),
+                                      "attention_only_frac_of_hbm": round(b_at / t_bat / 1e9 / hbm_peak, 4)},
                 "cached_candidates_by_batch": by_batch,
+                "kv_append": kv_append,
+                "block_stack": block,
                 "cached_serving": serving,
                 "beam_decode": beam,
                 "jagged_bf16": {"ms": round(jt / jsteps * 1e3, 4),
@@ -595,7 +779,7 @@ def run_gpu(args):
                          "achieved": round(a_attn_tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
                          "frac": round(a_attn_tflops / tf_peak, 4), "traffic": recorded_traffic(),
                          "peak_source": f"{peak_src} bf16 dense (burst)"},
-            "gpu_launches": args.steps * 9,
+            "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -629,10 +813,11 @@ def run_e2e(A, Bp, flush_buf, args):
     steps = max(3, min(args.steps, 5))
     flops, tot = 0.0, 0.0
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fa, _, _ = A.units()
+    fb, _, _ = Bp.units()
     for _ in range(steps):
+        A.reset(); Bp.reset()
         flush_buf.fill_(1)
-        fa, _, _ = A.units()
-        fb, _, _ = Bp.units()
         t0.record()
         for _, _, h, d in host:
             d.copy_(h, non_blocking=True)
@@ -748,6 +933,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks here (users are sharded by rank)
+        cmd = launcher_command(args.gpus, sys.argv[1:])
+        sys.exit(subprocess.call(cmd))
     if args.impl == "reference":
         run_reference(args)
     else:

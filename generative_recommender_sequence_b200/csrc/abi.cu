@@ -222,6 +222,7 @@ hstu_status hstu_attn_fwd(const void* q, const void* k, const void* v, const int
   p.scale = scale;
   p.max_q = p.max_kv = max_len;
   p.f32 = dt == HSTU_F32;
+  p.allow_split = false;  // no workspace: every item streams all of its keys
   return attn_dispatch(p, nullptr, 0, stream);
 }
 
@@ -391,26 +392,54 @@ static bool cached_problem(hstu_kv_table* t, const int64_t* users, int32_t B, co
 size_t hstu_attn_cached_workspace_size(hstu_kv_table* t, int32_t B, int64_t total_q, int32_t max_q,
                                        int32_t max_cached, int32_t mask_mode) {
   if (!t || B <= 0 || max_q <= 0 || t->dtype != HSTU_BF16 || t->dev.d != 128) return 0;
+  if (total_q <= 0 || max_cached < 0) return 0;
+  if (mask_mode != HSTU_MASK_CANDIDATES && mask_mode != HSTU_MASK_CAUSAL_SUFFIX) return 0;
   AttnProblem p;
   cached_problem(t, nullptr, B, nullptr, nullptr, nullptr, nullptr, total_q, max_q, max_cached,
                  mask_mode, &p);
   return attn_sm100_workspace_bytes(p, device_sm_count());
 }
 
+}  // extern "C"
+
+// Host-side argument checks of hstu_attn_cached_fwd (shared with its
+// allocation-free variant, so both report the same status for the same
+// arguments).  *nothing_to_do is set for a valid call with no query rows.
+hstu_status cached_fwd_validate(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
+                                const void* k_cand, const void* v_cand, const int64_t* q_offsets,
+                                int64_t total_q, int32_t max_q, int32_t max_cached,
+                                int32_t mask_mode, const hstu_rab* rab, const void* out,
+                                bool* nothing_to_do) {
+  *nothing_to_do = false;
+  if (!t || B < 0 || max_q < 0 || max_cached < 0 || total_q < 0) return HSTU_ERR_INVALID_ARG;
+  if (total_q >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
+  if (mask_mode != HSTU_MASK_CANDIDATES && mask_mode != HSTU_MASK_CAUSAL_SUFFIX)
+    return HSTU_ERR_INVALID_ARG;
+  if (B == 0 || max_q == 0 || total_q == 0) {
+    *nothing_to_do = true;
+    return HSTU_OK;
+  }
+  if (!users || !q || !q_offsets || !out) return HSTU_ERR_INVALID_ARG;
+  if (mask_mode == HSTU_MASK_CANDIDATES && (!k_cand || !v_cand)) return HSTU_ERR_INVALID_ARG;
+  if (mask_mode == HSTU_MASK_CAUSAL_SUFFIX && (k_cand || v_cand)) return HSTU_ERR_INVALID_ARG;
+  if (!rab_ok(rab, false)) return HSTU_ERR_UNSUPPORTED;
+  if (t->dtype == HSTU_BF16 && t->dev.d == 128 &&
+      (!aligned16(q) || !aligned16(out) || (k_cand && (!aligned16(k_cand) || !aligned16(v_cand)))))
+    return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+extern "C" {
+
 hstu_status hstu_attn_cached_fwd(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
                                  const void* k_cand, const void* v_cand, const int64_t* q_offsets,
                                  int64_t total_q, int32_t max_q, int32_t max_cached, int32_t mask_mode,
                                  const hstu_rab* rab, float scale, void* out, void* workspace,
                                  size_t ws_bytes, cudaStream_t stream) {
-  if (!t || B < 0 || max_q < 0 || max_cached < 0 || total_q < 0) return HSTU_ERR_INVALID_ARG;
-  if (total_q >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
-  if (mask_mode != HSTU_MASK_CANDIDATES && mask_mode != HSTU_MASK_CAUSAL_SUFFIX)
-    return HSTU_ERR_INVALID_ARG;
-  if (B == 0 || max_q == 0 || total_q == 0) return HSTU_OK;
-  if (!users || !q || !q_offsets || !out) return HSTU_ERR_INVALID_ARG;
-  if (mask_mode == HSTU_MASK_CANDIDATES && (!k_cand || !v_cand)) return HSTU_ERR_INVALID_ARG;
-  if (mask_mode == HSTU_MASK_CAUSAL_SUFFIX && (k_cand || v_cand)) return HSTU_ERR_INVALID_ARG;
-  if (!rab_ok(rab, false)) return HSTU_ERR_UNSUPPORTED;
+  bool nothing = false;
+  const hstu_status st = cached_fwd_validate(t, users, B, q, k_cand, v_cand, q_offsets, total_q,
+                                             max_q, max_cached, mask_mode, rab, out, &nothing);
+  if (st != HSTU_OK || nothing) return st;
   AttnProblem p;
   cached_problem(t, users, B, q, k_cand, v_cand, q_offsets, total_q, max_q, max_cached, mask_mode,
                  &p);
@@ -418,8 +447,6 @@ hstu_status hstu_attn_cached_fwd(hstu_kv_table* t, const int64_t* users, int32_t
   fill_rab(p, rab);
   p.scale = scale;
   if (!p.f32 && p.d == 128) {
-    if (!aligned16(q) || !aligned16(out) || (k_cand && (!aligned16(k_cand) || !aligned16(v_cand))))
-      return HSTU_ERR_INVALID_ARG;
     const size_t need = attn_sm100_workspace_bytes(p, device_sm_count());
     if (need > 0 && (workspace == nullptr || ws_bytes < need)) return HSTU_ERR_INVALID_ARG;
   }

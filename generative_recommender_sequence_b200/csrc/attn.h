@@ -42,6 +42,9 @@ struct AttnProblem {
   // write the unscaled fp32 partial sums of every key split to the workspace
   // and leave the reduction to the caller (no output, no split reduce)
   bool partial_only = false;
+  // callers without a workspace (hstu_attn_fwd, the uncached block) never
+  // split keys over CTAs
+  bool allow_split = true;
 };
 
 // bf16, d == 128, tcgen05 path.  workspace: fp32 split partials (may be null if

@@ -55,15 +55,12 @@ constexpr int VST = 2;             // V ring depth
 constexpr int kThreads = 640;      // 20 warps: TMA, MMA, timestamps, spare, 16 pointwise
 constexpr int kTileBytes = BM * HD * 2;   // 32 KiB
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
-constexpr int kPairHalfK = kHalfBytes / 2;  // CTA pair: one 64-column half of 64 keys
 constexpr int kMaxUsers = 1024;   // per launch; larger batches are split on the host
 constexpr int kMaxRab = 256;
 
 constexpr uint32_t TM_O = 0;      // O accumulator, 128 fp32 columns
 constexpr uint32_t TM_SP = 128;    // three S/P buffers of 128 columns each
 constexpr int NSP = 3;
-// whether eligible launches use CTA pairs when HSTU_ATTN_CTA_PAIRS is unset
-constexpr bool kCtaPairsByDefault = false;
 // P (bf16 pairs) overwrites the first half of each pointwise warp's own S
 // columns.  16 warps per tile (32 columns each): keys [32 c, 32 c + 32) ->
 // columns [32 c, 32 c + 16), so MMA k-step kk (16 keys) starts at column
@@ -77,9 +74,6 @@ __host__ __device__ constexpr uint32_t p_col(int kk) {
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
-// CTA pair: M = 256 rows over the two CTAs, each supplying half of B's N columns
-constexpr uint32_t kIdescQK2 = idesc_bf16_f32(2 * BM, BN, false);
-constexpr uint32_t kIdescPV2 = idesc_bf16_f32(2 * BM, HD, true);
 
 constexpr int NTS = 4;              // key-timestamp ring depth
 constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
@@ -114,10 +108,9 @@ struct __align__(1024) Smem {
   uint64_t q_full[QST], q_empty[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  // s_full per (pair, buffer) = tile index mod 6, so each pair waits every phase
-  // of its own barriers in order; p_full / sp_empty have one in-order waiter
   // s_full: one per buffer (16-warp layout) or per (pair, buffer) = tile mod 6
-  // (two-pair layout), so each waiter sees every phase of its barriers in order
+  // (two-pair layout), so each waiter sees every phase of its barriers in order;
+  // p_full / sp_empty have one in-order waiter
   uint64_t s_full[2 * NSP], p_full[NSP], sp_empty[NSP];
   uint64_t o_full[2], o_empty;  // o_full[1]: second pair of the two-pair layout
   uint64_t ts_full[NTS], ts_empty[NTS];
@@ -125,10 +118,18 @@ struct __align__(1024) Smem {
   uint64_t mma_done, mma_done2;
   uint32_t tmem_base;
   int abort_flag;
+  // balanced key splits: this CTA's one item (valid, user, query tile, head,
+  // key-tile range), derived by plan_balanced
+  int bal_ok, bal_b, bal_m, bal_h, bal_t0, bal_t1;
 };
 
 struct KParams {
   int B, H, mode, n_split, kps;
+  // balanced key splits: per-user split counts chosen on the device, one item
+  // per CTA; partial sums of item t at partial + t * BM * HD, and the item
+  // offsets per user (int32 [B + 1]) written to plan for the reduce
+  int balanced;
+  int* plan;
   const int64_t* q_off;
   const int64_t* kv_off;
   const int64_t* users;
@@ -216,14 +217,12 @@ struct Sched {
   }
 };
 
-// Items are sorted longest first; round k hands them to the CTAs (CTA pairs
-// when PAIR) in forward order for even k and in reverse order for odd k (a
-// snake), so the one that got the longest item of a round gets the shortest of
-// the next.
-template <bool PAIR>
+// Items are sorted longest first; round k hands them to the CTAs in forward
+// order for even k and in reverse order for odd k (a snake), so the CTA that
+// got the longest item of a round gets the shortest of the next.
 __device__ __forceinline__ long long snake_item(long long rnd) {
-  const long long G = gridDim.x >> (PAIR ? 1 : 0);
-  const long long me = blockIdx.x >> (PAIR ? 1 : 0);
+  const long long G = gridDim.x;
+  const long long me = blockIdx.x;
   return rnd * G + ((rnd & 1) ? (G - 1 - me) : me);
 }
 
@@ -239,22 +238,18 @@ struct Item {
   int t0, t1;       // this item's tile range
 };
 
-// Item m of user b covers query rows [bm m, bm m + bm) with bm = BM, or, for a
-// CTA pair, bm = 2 BM rows of which CTA `rank` owns [bm m + BM rank, + BM).
-// Both CTAs of a pair derive the same key-tile range (that of the whole block);
-// rows of the lower half simply see more fully masked tiles.
-template <bool PAGED, bool CAND, bool PAIR>
-__device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem,
-                                          uint32_t rank) {
+// Item m of user b covers query rows [BM m, BM m + BM).
+template <bool PAGED, bool CAND>
+__device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem) {
   Item it;
   it.b = b;
   it.m = m;
   it.h = rem / P.n_split;
   it.s = rem % P.n_split;
-  const int64_t bm = PAIR ? 2 * BM : BM;
+  const int64_t bm = BM;
   const int64_t qs = sm.m_q[b], nq = (int64_t)sm.m_q[b + 1] - qs;
   const int64_t blk0 = bm * m;                           // first row of the block
-  const int64_t r0 = blk0 + (PAIR ? (int64_t)BM * rank : 0);  // first row of this CTA
+  const int64_t r0 = blk0;
   it.q_row0 = qs + r0;
   it.nvalid = (int)max64(0, min64(BM, nq - r0));
   it.n_k = sm.m_nk[b];
@@ -277,7 +272,11 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
     it.n_main = last >= 0 ? (int)(last / BN) + 1 : 0;
     total = it.n_main;
   }
-  if (P.n_split > 1) {
+  if (P.balanced) {
+    it.s = blockIdx.x;  // the item id: where its partial sums go
+    it.t0 = sm.bal_t0;
+    it.t1 = min(total, sm.bal_t1);
+  } else if (P.n_split > 1) {
     it.t0 = it.s * P.kps;
     it.t1 = min(total, it.t0 + P.kps);
   } else {
@@ -287,26 +286,116 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
   return it;
 }
 
-// MMA completion: one CTA's barrier, or the same barrier in both CTAs of a pair.
-template <bool PAIR>
-__device__ __forceinline__ void commit(uint32_t bar) {
-  if (PAIR)
-    umma_commit_pair(bar);
-  else
-    umma_commit(bar);
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
-// Arrive on a barrier that CTA 0 of a pair owns (this CTA's own otherwise).
-template <bool PAIR>
-__device__ __forceinline__ void arrive_shared(uint32_t bar) {
-  if (PAIR)
-    mbar_arrive_cluster(mapa_shared(bar, 0));
-  else
-    mbar_arrive(bar);
+
+// Key tiles of one query tile of user b (the same for every query tile of a
+// candidate user; causal runs in this mode have at most one query tile) and
+// its number of query tiles.
+template <bool CAND>
+__device__ __forceinline__ int plan_tiles(const KParams& P, const Smem& sm, int b, int& qt) {
+  const int nq = sm.m_q[b + 1] - sm.m_q[b];
+  const int64_t n_k = sm.m_nk[b];
+  qt = nq > 0 ? (nq + BM - 1) / BM : 0;
+  if (qt == 0) return 0;
+  if (CAND) return (int)((n_k + BN - 1) / BN) + 1;
+  const int64_t last = n_k - nq + min64(BM, nq) - 1;
+  return last >= 0 ? (int)(last / BN) + 1 : 0;
 }
-// Wait on a barrier that both CTAs of a pair arrive on.
-template <bool PAIR>
-__device__ __forceinline__ bool wait_shared(uint32_t bar, uint32_t parity) {
-  return PAIR ? mbar_wait_cluster(bar, parity) : mbar_wait(bar, parity);
+
+// Runs a user's key tiles are cut into for a target run length (round to
+// nearest, at least one run, never more runs than tiles).
+__device__ __forceinline__ int plan_runs(int tiles, int target) {
+  if (tiles <= 0) return 0;
+  return max(1, min(tiles, (tiles + target / 2) / target));
+}
+
+// Balanced key splits (candidate scoring and short causal runs, when there are
+// fewer (user, head, query tile) items than CTAs).  Every CTA derives the same
+// plan from the key counts: the target run length is the smallest that is at
+// least ceil(total tiles / CTAs) and lets every user's runs fit one wave, user
+// b's tiles are cut into plan_runs(tiles_b, target) near-equal runs, and items
+// are numbered user by user, then query tile, head and run.  This CTA takes
+// item blockIdx.x; CTA 0 also publishes each user's first item for the reduce.
+// Called by warp 0 only.
+template <bool CAND>
+__device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
+  const int G = gridDim.x;
+  long long W = 0;
+  for (int b0 = 0; b0 < P.B; b0 += 32) {
+    const int b = b0 + lane;
+    int qt = 0;
+    const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
+    W += (long long)qt * P.H * t;
+  }
+  W = warp_sum_ll(W);
+  int target = (int)max(2LL, (W + G - 1) / G);
+  for (int iter = 0;; ++iter) {
+    long long items = 0;
+    for (int b0 = 0; b0 < P.B; b0 += 32) {
+      const int b = b0 + lane;
+      int qt = 0;
+      const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
+      items += (long long)qt * P.H * plan_runs(t, target);
+    }
+    items = warp_sum_ll(items);
+    if (items <= G) break;
+    // one run per user always fits (the host chooses this mode only then)
+    target = iter < 64 ? target + 1 : (1 << 30);
+  }
+  // this CTA's item: exclusive prefix of the users' item counts
+  const long long me = blockIdx.x;
+  long long base = 0;
+  bool found = false;
+  if (lane == 0) sm.bal_ok = 0;
+  __syncwarp();
+  for (int b0 = 0; b0 < P.B; b0 += 32) {
+    const int b = b0 + lane;
+    int qt = 0;
+    const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
+    const int ns = plan_runs(t, target);
+    const long long cnt = (long long)qt * P.H * ns;
+    long long incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const long long first = base + incl - cnt;
+    if (blockIdx.x == 0 && b < P.B) P.plan[b] = (int)first;
+    if (b < P.B && cnt > 0 && me >= first && me < first + cnt) {
+      const int r = (int)(me - first);
+      const int per = P.H * ns;
+      const int h = (r % per) / ns, sidx = r % ns;
+      sm.bal_b = b;
+      sm.bal_m = r / per;
+      sm.bal_h = h;
+      sm.bal_t0 = (int)((long long)sidx * t / ns);
+      sm.bal_t1 = (int)((long long)(sidx + 1) * t / ns);
+      sm.bal_ok = 1;
+      found = true;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (blockIdx.x == 0 && lane == 0) P.plan[P.B] = (int)base;
+  (void)found;
+}
+
+// The rnd-th item of this CTA: one fixed item with balanced splits, otherwise
+// the snake order over the longest-first item list.
+__device__ __forceinline__ bool next_item(const KParams& P, const Smem& sm, Sched<BM>& sc,
+                                          long long rnd, int lane, int& b, int& m, int& rem) {
+  if (P.balanced) {
+    if (rnd > 0 || !sm.bal_ok) return false;
+    b = sm.bal_b;
+    m = sm.bal_m;
+    rem = sm.bal_h;
+    return true;
+  }
+  return sc.item(snake_item(rnd), sm.m_q, lane, b, m, rem);
 }
 
 __device__ __forceinline__ void record_timeout(const KParams& P, Smem& sm) {
@@ -419,7 +508,7 @@ __device__ __forceinline__ void pw_chunk_any(const uint32_t (&sv)[16], uint32_t 
 }
 
 // ------------------------------------------------------------ the kernel
-template <bool PAGED, bool CAND, bool PAIR, bool PW2>
+template <bool PAGED, bool CAND, bool PW2>
 __global__ void __launch_bounds__(kThreads, 1)
     hstu_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -429,12 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
-  static_assert(!(PAIR && CAND), "CTA pairs serve the causal path only");
-  static_assert(!(PAIR && PW2), "CTA pairs use the 16-warp pointwise layout");
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  // rank in the CTA pair (0 issues the pair's MMAs and owns the shared barriers)
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   // dependent launch: the next kernel may start being scheduled.  Barrier
   // initialisation, the descriptor prefetch and the TMEM allocation touch no
   // global memory, so they overlap the previous kernel's tail; every global
@@ -456,8 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.v_empty[i]), 1);
     }
     // P written / O drained: the warps that handle a tile (16, or one pair of
-    // 8 in the two-pair layout), of each CTA of a CTA pair
-    constexpr uint32_t kTileWarps = PW2 ? 8 : (PAIR ? 32 : 16);
+    // 8 in the two-pair layout)
+    constexpr uint32_t kTileWarps = PW2 ? 8 : 16;
     for (int i = 0; i < 2 * NSP; ++i) mbar_init(smem_u32(&sm.s_full[i]), 1);
     for (int i = 0; i < NSP; ++i) {
       mbar_init(smem_u32(&sm.p_full[i]), kTileWarps);
@@ -486,13 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(smem_u32(&sm.tmem_base), 512);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(&sm.tmem_base), 512);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
   }
   pdl_wait();
 
@@ -504,6 +584,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // an out-of-range user id has no cached tokens (and no page list is read)
       const int64_t u = P.users[b];
       const bool known = u >= 0 && u < P.max_users;
+      if (known) {
+        // the producer reads this user's page ids once the items are known:
+        // start them towards L2 now, beside the length load
+        const int32_t* pl = P.page_lists + u * (int64_t)P.max_ppu;
+        const int n = min(P.max_ppu, kPagesStaged);
+        for (int i = 0; i < n; i += 32) prefetch_l2(pl + i);
+      }
       sm.m_kv[b] = known ? (int)u : 0;
       sm.m_nk[b] = known ? (int)P.lengths[u] : 0;
     } else {
@@ -515,43 +602,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.pos_ext[i] = P.pos_table ? P.pos_table[min(i, P.n_pos - 1)] : 0.f;
     sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
   }
+  __syncthreads();
+  if (P.balanced && warp == 0) plan_balanced<CAND>(P, sm, lane);
   tc_fence_before();
   __syncthreads();
-  // the peer CTA signals barriers of CTA 0 only after both have initialised them
-  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int HS = P.H * P.n_split;
 
   if (warp == 0) {
     // =============================================== TMA producer
-    Sched<PAIR ? 2 * BM : BM> sc;
+    Sched<BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
-      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
         const uint32_t qs = qi % QST;
         ok = mbar_wait(smem_u32(&sm.q_empty[qs]), ((qi / QST) & 1) ^ 1);
         if (ok) {
           const uint32_t bar = smem_u32(&sm.q_full[qs]);
-          if (PAIR) {
-            // each CTA loads its own 128 rows; CTA 0's barrier counts both
-            const uint32_t lbar = mapa_shared(bar, 0);
-            if (rank == 0) mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-            tma_load_3d_pair(smem_u32(sm.q[qs]), &tm_q, lbar, 0, it.h, (int)it.q_row0);
-            tma_load_3d_pair(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, lbar, 64, it.h,
-                             (int)it.q_row0);
-          } else {
-            mbar_arrive_expect_tx(bar, kTileBytes);
-            tma_load_3d(smem_u32(sm.q[qs]), &tm_q, bar, 0, it.h, (int)it.q_row0);
-            tma_load_3d(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
-          }
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          tma_load_3d(smem_u32(sm.q[qs]), &tm_q, bar, 0, it.h, (int)it.q_row0);
+          tma_load_3d(smem_u32(sm.q[qs]) + kHalfBytes, &tm_q, bar, 64, it.h, (int)it.q_row0);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -588,34 +665,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = smem_u32(which == 0 ? sm.k[slot] : sm.v[slot]);
           if (lane == 0) {
             ok = mbar_wait(smem_u32(which == 0 ? &sm.k_empty[slot] : &sm.v_empty[slot]), par);
-            // a pair's tile is two 16 KiB halves, one per CTA, counted by CTA 0
-            if (ok && (!PAIR || rank == 0)) mbar_arrive_expect_tx(bar, kTileBytes);
+            if (ok) mbar_arrive_expect_tx(bar, kTileBytes);
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           if (which == 0) ++kc; else ++vc;
           const int half = lane & 1;
-          if (PAIR) {
-            // K: keys [64 rank, 64 rank + 64) of the tile (pages 2 rank, 2 rank + 1),
-            //    both 64-column halves, as a 64-row K-major block per half;
-            // V: all four pages, value columns [64 rank, 64 rank + 64).
-            if (lane < 4) {
-              const int pg = which == 0 ? 2 * (int)rank + (lane >> 1) : lane;
-              const int idx = tile * 4 + pg;
-              const int si = (tile - it.t0) * 4 + pg;
-              const int32_t* plist = P.page_lists + it.user * (int64_t)P.max_ppu;
-              int64_t page = si < kPagesStaged ? (int64_t)sm.pages[si]
-                                               : (idx < P.max_ppu ? (int64_t)plist[idx] : -1);
-              if (page < 0 || page >= P.n_pages) page = P.n_pages;  // the zero page
-              const int row = (int)(((page * 2 + which) * P.H + it.h) * 32);
-              const uint32_t lbar = mapa_shared(bar, 0);
-              if (which == 0)
-                tma_load_2d_pair(dst + half * kPairHalfK + (lane >> 1) * 4096, &tm_k, lbar,
-                                 half * 64, row);
-              else
-                tma_load_2d_pair(dst + lane * 4096, &tm_k, lbar, 64 * (int)rank, row);
-            }
-          } else if (CAND && tile == it.n_main) {
+          if (CAND && tile == it.n_main) {
             if (lane < 2)
               tma_load_3d(dst + half * kHalfBytes, which == 0 ? &tm_kc : &tm_vc, bar, half * 64,
                           it.h, (int)it.q_row0);
@@ -640,14 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-    if (!ok && lane == 0 && PAIR && rank != 0) {
-      // this CTA's copies signal CTA 0's barriers, which it cannot wait on:
-      // give any copy still in flight time to land before the CTA can exit
-      record_timeout(P, sm);
-      const unsigned long long t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 200000ull) {
-      }
-    } else if (!ok && lane == 0) {
+    if (!ok && lane == 0) {
       record_timeout(P, sm);
       // let copies already in flight land before the CTA can exit
       for (uint32_t i = 0; i < KST && i < kc; ++i) {
@@ -667,17 +716,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =============================================== MMA issuers
     // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
     // tensor pipe fed: while one waits on its barriers the other's MMAs run.
-    Sched<PAIR ? 2 * BM : BM> sc;
+    Sched<BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
-    // in a CTA pair only CTA 0 issues (M = 256 MMAs over both CTAs' operands)
-    for (long long rnd = 0; ok && (!PAIR || rank == 0); ++rnd) {
-      const long long t = snake_item<PAIR>(rnd);
+    for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       const int nt = it.t1 - it.t0;
       if (lane == 0) {
@@ -698,28 +745,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < HD / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
               const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-              if (PAIR) {
-                // each CTA holds 64 keys: 64-row blocks per 64-column half
-                const uint32_t koff = (kk >> 2) * kPairHalfK + (kk & 3) * 32;
-                const uint64_t bdesc = smem_desc_sw128(k_base + koff, 16, 1024);
-                umma_ss_pair(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK2, kk > 0 ? 1u : 0u);
-              } else {
-                const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-                umma_ss(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
-              }
+              const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+              umma_ss(tmem + TM_SP + sb * 128, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
             }
-            commit<PAIR>(smem_u32(&sm.k_empty[slot]));
-            commit<PAIR>(smem_u32(&sm.s_full[PW2 ? g % (2 * NSP) : sb]));
-            if (i == nt - 1) commit<PAIR>(smem_u32(&sm.q_empty[qs]));
+            umma_commit(smem_u32(&sm.k_empty[slot]));
+            umma_commit(smem_u32(&sm.s_full[PW2 ? g % (2 * NSP) : sb]));
+            if (i == nt - 1) umma_commit(smem_u32(&sm.q_empty[qs]));
           }
         } else {
           for (int i = 0; i < nt && ok; ++i, ++g, ++vc) {
             const uint32_t pb = g % NSP;
             const uint32_t slot = vc % VST;
-            // P and drained-O arrivals come from both CTAs of a pair
-            ok = wait_shared<PAIR>(smem_u32(&sm.p_full[pb]), (g / NSP) & 1) &&
+            ok = mbar_wait(smem_u32(&sm.p_full[pb]), (g / NSP) & 1) &&
                  mbar_wait(smem_u32(&sm.v_full[slot]), (vc / VST) & 1) &&
-                 (i != 0 || wait_shared<PAIR>(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
+                 (i != 0 || mbar_wait(smem_u32(&sm.o_empty), (qi & 1) ^ 1));
             if (!ok) break;
             tc_fence_after();
             const uint32_t v_base = smem_u32(sm.v[slot]);
@@ -727,31 +766,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BN / 16; ++kk) {
               // V tile is MN-major: 64-column halves 16 KiB apart (LBO), 8-key
               // groups 1 KiB apart (SBO); 16 keys = 2 KiB per k-step.
-              // (a CTA of a pair holds one 64-column half: the same layout)
               const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
-              if (PAIR)
-                umma_ts_pair(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col<PW2>(kk), bdesc, kIdescPV2,
-                             (i == 0 && kk == 0) ? 0u : 1u);
-              else
-                umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col<PW2>(kk), bdesc, kIdescPV,
-                        (i == 0 && kk == 0) ? 0u : 1u);
+              umma_ts(tmem + TM_O, tmem + TM_SP + pb * 128 + p_col<PW2>(kk), bdesc, kIdescPV,
+                      (i == 0 && kk == 0) ? 0u : 1u);
             }
-            commit<PAIR>(smem_u32(&sm.v_empty[slot]));
-            commit<PAIR>(smem_u32(&sm.sp_empty[pb]));
+            umma_commit(smem_u32(&sm.v_empty[slot]));
+            umma_commit(smem_u32(&sm.sp_empty[pb]));
           }
           // two-pair layout: the pair that took the item's last key tile runs its epilogue
-          if (ok) commit<PAIR>(smem_u32(&sm.o_full[PW2 ? (g - 1) & 1 : 0]));
+          if (ok) umma_commit(smem_u32(&sm.o_full[PW2 ? (g - 1) & 1 : 0]));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       g = __shfl_sync(0xffffffffu, g, 0);
       ++qi;
     }
-    if (lane == 0 && (!PAIR || rank == 0)) {
+    if (lane == 0) {
       if (!ok) record_timeout(P, sm);
       // all MMAs issued by this thread must finish before TMEM is released
       const uint32_t done = smem_u32(qk_role ? &sm.mma_done : &sm.mma_done2);
-      commit<PAIR>(done);
+      umma_commit(done);
       mbar_wait(done, 0);
     }
     __syncwarp();
@@ -760,15 +794,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Stages the key timestamps of every tile (in the MMA's tile order) for the
     // time-gap bias, so the pointwise warps never wait on global loads.
     if (P.time_table != nullptr && !PAGED && !CAND) {
-      Sched<PAIR ? 2 * BM : BM> sc;
+      Sched<BM> sc;
       sc.init(sm.m_q, P.B, HS, lane);
       uint32_t g = 0, qitem = 0;
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item<PAIR>(rnd);
         int b, m, rem;
-        if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-        const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+        if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
+        const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
         if (it.t0 >= it.t1) continue;
         const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
         {  // query timestamps of this item's rows
@@ -855,15 +888,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rarely touched on the constant-row path)
     int pb_idx = -1;
     float pb_val = 0.f;
-    Sched<PAIR ? 2 * BM : BM> sc;
+    Sched<BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     uint32_t qi = 0, g = 0, my_epi = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
@@ -1001,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.p_full[sb]));
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       }
       if (!ok) break;
       if (use_time) {
@@ -1033,14 +1065,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q == 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.o_empty));
+          if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
         }
         if (!row_ok) continue;
         if (P.partial) {
           // whole 32-byte sectors when the buffer allows: the scattered
           // per-row partial stores drain faster than as 16-byte pieces
-          float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
-                       it.h * HD + ocol;
+          float* dst = P.balanced
+                           ? P.partial + ((int64_t)it.s * BM + r) * HD + ocol
+                           : P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
+                                 it.h * HD + ocol;
           if (P.part_v8) {
 #pragma unroll
             for (int j = 0; j < 32; j += 8) st_global_v8(dst + j, oa + j);
@@ -1091,15 +1125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rarely touched on the constant-row path)
     int pb_idx = -1;
     float pb_val = 0.f;
-    Sched<PAIR ? 2 * BM : BM> sc;
+    Sched<BM> sc;
     sc.init(sm.m_q, P.B, HS, lane);
     uint32_t qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
-      const long long t = snake_item<PAIR>(rnd);
       int b, m, rem;
-      if (!sc.item(t, sm.m_q, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND, PAIR>(P, sm, b, m, rem, rank);
+      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
@@ -1215,7 +1248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.p_full[sb]));
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       }
       if (!ok) break;
       if (use_time) {
@@ -1235,13 +1268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence(oa);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_shared<PAIR>(smem_u32(&sm.o_empty));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
       if (row_ok) {
         if (P.partial) {
           // whole 32-byte sectors when the buffer allows: the scattered
           // per-row partial stores drain faster than as 16-byte pieces
-          float* dst = P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
-                       it.h * HD + cbase;
+          float* dst = P.balanced
+                           ? P.partial + ((int64_t)it.s * BM + r) * HD + cbase
+                           : P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
+                                 it.h * HD + cbase;
           if (P.part_v8) {
 #pragma unroll
             for (int j = 0; j < 32; j += 8) st_global_v8(dst + j, oa + j);
@@ -1274,15 +1309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
-  // a pair's MMAs write both CTAs' tensor memory and each CTA signals the
-  // other's barriers: neither releases anything before both are done
-  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR)
-      tmem_dealloc_pair(tmem, 512);
-    else
-      tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1293,7 +1322,9 @@ __global__ void split_reduce_kernel(KParams P, int B) {
   pdl_launch_dependents();
   pdl_wait();
   const int64_t row = blockIdx.x;
-  if (row >= P.total_q || row >= P.q_off[B]) return;
+  // a launch for one chunk of users owns rows [q_off[0], q_off[B]) only: rows of
+  // other chunks are finished outputs and must not be touched
+  if (row >= P.total_q || row < P.q_off[0] || row >= P.q_off[B]) return;
   // find the user of this row
   int lo = 0, hi = B;
   while (hi - lo > 1) {
@@ -1302,6 +1333,35 @@ __global__ void split_reduce_kernel(KParams P, int B) {
     else hi = mid;
   }
   const int b = lo;
+  const int F = P.H * HD;
+  if (P.balanced) {
+    // item (user b, query tile m, head h, run s) = plan[b] + (m H + h) ns + s
+    const int64_t rel = row - P.q_off[b];
+    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
+    const int qt = (int)((nq + BM - 1) / BM);
+    const int m = (int)(rel / BM), rr = (int)(rel % BM);
+    const int first = P.plan[b];
+    const int ns = (P.plan[b + 1] - first) / (qt * P.H);
+    for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
+      const int h = f / HD, c = f % HD;
+      const int item0 = first + (m * P.H + h) * ns;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sidx = 0; sidx < ns; ++sidx) {
+        const float4 x = *reinterpret_cast<const float4*>(
+            P.partial + ((int64_t)(item0 + sidx) * BM + rr) * HD + c);
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+      }
+      __nv_bfloat16* dst = P.out + row * P.out_stride + f;
+      uint2 u;
+      u.x = pack_bf16x2(acc.x * P.scale, acc.y * P.scale);
+      u.y = pack_bf16x2(acc.z * P.scale, acc.w * P.scale);
+      *reinterpret_cast<uint2*>(dst) = u;
+    }
+    return;
+  }
   int64_t n_k;
   if (PAGED) {
     const int64_t u = P.users[b];
@@ -1320,7 +1380,6 @@ __global__ void split_reduce_kernel(KParams P, int B) {
     total = last >= 0 ? (int)(last / BN) + 1 : 0;
   }
   const int n_valid = min(P.n_split, (total + P.kps - 1) / P.kps);
-  const int F = P.H * HD;
   for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < n_valid; ++s) {
@@ -1340,7 +1399,7 @@ __global__ void split_reduce_kernel(KParams P, int B) {
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-template <bool PAGED, bool CAND, bool PAIR, bool PW2 = false>
+template <bool PAGED, bool CAND, bool PW2 = false>
 cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items, int num_sms,
                         cudaStream_t stream) {
   CUtensorMap tq, tk, tv, tkc, tvc;
@@ -1367,9 +1426,8 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     tkc = tq;
     tvc = tq;
   }
-  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PAIR, PW2>;
+  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PW2>;
   static bool attr_set[64] = {};
-  static int max_pairs[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   const bool cached = dev >= 0 && dev < 64 && attr_set[dev];
@@ -1377,53 +1435,14 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes());
     if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  cudaError_t e;
-  if (!PAIR) {
-    const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
-    if (!cached && dev >= 0 && dev < 64) attr_set[dev] = true;
-    e = launch_dependent(kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq, tk, tv, tkc,
-                         tvc, kp);
-  } else {
-    // persistent CTA pairs: as many 2-CTA clusters as can be resident at once
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes();
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int pairs = cached ? max_pairs[dev] : 0;
-    if (!cached) {
-      cfg.gridDim = dim3(2 * (unsigned)std::max(1, num_sms / 2));
-      if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs <= 0) {
-        cudaGetLastError();
-        pairs = std::max(1, num_sms / 2);
-      }
-      if (dev >= 0 && dev < 64) {
-        max_pairs[dev] = pairs;
-        attr_set[dev] = true;
-      }
-    }
-    const long long n = std::max<long long>(1, std::min<long long>(items, pairs));
-    cfg.gridDim = dim3(2 * (unsigned)n);
-    e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tkc, tvc, kp);
-    if (e == cudaSuccess) e = cudaGetLastError();
-  }
+  const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
+  cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq, tk,
+                                   tv, tkc, tvc, kp);
   if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
   return launch_dependent(split_reduce_kernel<PAGED>, dim3((unsigned)p.total_q), dim3(128), 0, stream,
                           kp, p.B);
-}
-
-// -1 when HSTU_ATTN_CTA_PAIRS is unset, else 0 / 1.
-int cta_pair_override() {
-  const char* e = std::getenv("HSTU_ATTN_CTA_PAIRS");
-  if (e == nullptr || *e == 0) return -1;
-  return std::atoi(e) != 0 ? 1 : 0;
 }
 
 // Key-split plan: one wave of (user, head, split) items, each streaming a long
@@ -1433,6 +1452,7 @@ int cta_pair_override() {
 void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
   *n_split = 1;
   *kps = 1 << 30;
+  if (!p.allow_split && !p.partial_only) return;
   if (p.mode != 1 && p.max_q > BM) return;
   const int max_tiles = (p.max_kv + BN - 1) / BN + (p.mode == 1 ? 1 : 0);
   const int qt = std::max(1, (p.max_q + BM - 1) / BM);
@@ -1450,6 +1470,8 @@ void split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
   }
 }
 
+size_t balanced_plan_bytes(int B) { return ((size_t)(B + 1) * sizeof(int) + 255) & ~size_t(255); }
+
 }  // namespace
 
 void attn_sm100_split_plan(const AttnProblem& p, int num_sms, int* n_split, int* kps) {
@@ -1457,9 +1479,28 @@ void attn_sm100_split_plan(const AttnProblem& p, int num_sms, int* n_split, int*
 }
 
 size_t attn_sm100_workspace_bytes(const AttnProblem& p, int num_sms) {
+  if (p.B > kMaxUsers) {
+    // batches over kMaxUsers run as chunks of users (attn_sm100_launch), each
+    // with its own key-split plan over the same absolute query rows: the
+    // workspace must hold the largest chunk's partials.  A short last chunk
+    // can split keys where a full one does not.
+    AttnProblem c = p;
+    c.B = kMaxUsers;
+    size_t need = attn_sm100_workspace_bytes(c, num_sms);
+    if (p.B % kMaxUsers != 0) {
+      c.B = p.B % kMaxUsers;
+      need = std::max(need, attn_sm100_workspace_bytes(c, num_sms));
+    }
+    return need;
+  }
   int ns, kps;
   split_plan(p, num_sms, &ns, &kps);
   if (ns <= 1 && !p.partial_only) return 0;
+  if (!p.partial_only) {
+    // balanced splits: the per-user item offsets, then one fp32 [BM, HD] block
+    // per item, at most one item per SM
+    return balanced_plan_bytes(p.B) + (size_t)num_sms * BM * HD * sizeof(float);
+  }
   return (size_t)ns * (size_t)p.total_q * p.H * HD * sizeof(float);
 }
 
@@ -1506,30 +1547,35 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
   kp.out_stride = p.out_stride;
   kp.total_q = p.total_q;
   kp.err = err_word;
+  long long items_override = -1;
   if (kp.n_split > 1 || p.partial_only) {
     const size_t need = attn_sm100_workspace_bytes(p, num_sms);
     if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
-    kp.partial = reinterpret_cast<float*>(workspace);
-    kp.part_v8 = (reinterpret_cast<uintptr_t>(workspace) & 31) == 0 ? 1 : 0;
+    if (!p.partial_only) {
+      // balanced splits, one item per CTA (the kernel chooses the runs)
+      kp.balanced = 1;
+      kp.n_split = 1;
+      kp.kps = 1 << 30;
+      kp.plan = reinterpret_cast<int*>(workspace);
+      kp.partial = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                            balanced_plan_bytes(p.B));
+      items_override = num_sms;
+    } else {
+      kp.partial = reinterpret_cast<float*>(workspace);
+    }
+    kp.part_v8 = (reinterpret_cast<uintptr_t>(kp.partial) & 31) == 0 ? 1 : 0;
   }
-  // Paged causal attention over long query runs may go to CTA pairs: each pair
-  // shares every K/V tile (each CTA loads half), halving the tile traffic into
-  // shared memory per SM.  HSTU_ATTN_CTA_PAIRS=1 / 0 forces the choice.
-  const bool eligible = p.paged && p.mode != 1 && p.max_q >= 2 * BM;
-  const int forced = cta_pair_override();
-  const bool pair = eligible && (forced >= 0 ? forced == 1 : kCtaPairsByDefault);
-  const int bm = pair ? 2 * BM : BM;
-  const int qt = (p.max_q + bm - 1) / bm;
-  const long long items = (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
+  const int qt = (p.max_q + BM - 1) / BM;
+  const long long items =
+      items_override > 0 ? items_override : (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
   if (p.paged) {
-    if (p.mode == 1) return launch_impl<true, true, false>(p, kp, items, num_sms, stream);
+    if (p.mode == 1) return launch_impl<true, true>(p, kp, items, num_sms, stream);
     // paged causal attention (the long-history path) runs the two-pair
     // pointwise layout: measured faster there than 16 warps per tile
-    return pair ? launch_impl<true, false, true>(p, kp, items, num_sms, stream)
-                : launch_impl<true, false, false, true>(p, kp, items, num_sms, stream);
+    return launch_impl<true, false, true>(p, kp, items, num_sms, stream);
   }
-  return p.mode == 1 ? launch_impl<false, true, false>(p, kp, items, num_sms, stream)
-                     : launch_impl<false, false, false>(p, kp, items, num_sms, stream);
+  return p.mode == 1 ? launch_impl<false, true>(p, kp, items, num_sms, stream)
+                     : launch_impl<false, false>(p, kp, items, num_sms, stream);
 }
 
 }  // namespace hstu

@@ -359,6 +359,7 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
     a.ts = p.ts;
     a.scale = p.scale;
     a.max_q = a.max_kv = p.max_len;
+    a.allow_split = false;  // the block's workspace holds no split partials
     e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
     if (e != cudaSuccess) return e;
     e = launch_dependent(ln_gate_kernel, dim3((unsigned)((p.T + 7) / 8)), dim3(256), 0, stream,

@@ -13,7 +13,9 @@
 //  - host code never uses the array's name as an address: the first call on
 //    each device (with that device current) asks cudaGetSymbolAddress for it
 //    and caches the result, so that first call should happen before any
-//    stream capture begins;
+//    stream capture begins.  The cache assumes the device's primary context
+//    lives as long as the process (no cudaDeviceReset in between, which would
+//    also invalidate every KV table);
 //  - a call whose partial sums would not fit returns HSTU_ERR_UNSUPPORTED;
 //  - every call shares the array and it keeps the last call's contents.  No
 //    part of it has to start at zero (each partial is written before it is
@@ -27,6 +29,15 @@
 
 #include "../../include/hstu.h"
 #include "attn.h"
+
+// The argument checks of hstu_attn_cached_fwd (abi.cu): this entry point runs
+// them before sizing its scratch, so both report the same status for the same
+// arguments.
+hstu_status cached_fwd_validate(hstu_kv_table* t, const int64_t* users, int32_t B, const void* q,
+                                const void* k_cand, const void* v_cand, const int64_t* q_offsets,
+                                int64_t total_q, int32_t max_q, int32_t max_cached,
+                                int32_t mask_mode, const hstu_rab* rab, const void* out,
+                                bool* nothing_to_do);
 
 namespace {
 
@@ -62,7 +73,10 @@ hstu_status hstu_attn_cached_fwd_noalloc(hstu_kv_table* t, const int64_t* users,
                                          int32_t max_cached, int32_t mask_mode,
                                          const hstu_rab* rab, float scale, void* out,
                                          cudaStream_t stream) {
-  if (!t) return HSTU_ERR_INVALID_ARG;
+  bool nothing = false;
+  const hstu_status st = cached_fwd_validate(t, users, B, q, k_cand, v_cand, q_offsets, total_q,
+                                             max_q, max_cached, mask_mode, rab, out, &nothing);
+  if (st != HSTU_OK || nothing) return st;
   const size_t need =
       hstu_attn_cached_workspace_size(t, B, total_q, max_q, max_cached, mask_mode);
   if (need > kNoAllocScratchBytes) return HSTU_ERR_UNSUPPORTED;

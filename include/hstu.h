@@ -264,9 +264,12 @@ HSTU_API size_t hstu_attn_cached_workspace_size(hstu_kv_table* t, int32_t B, int
  * that the library reserves on every GPU where it is loaded, kept until the
  * process exits.  Calls needing more than that return HSTU_ERR_UNSUPPORTED.
  * The first call on a device looks the array's address up (with that device
- * current) and should come before any stream capture.  All calls share the
+ * current) and should come before any stream capture; the address is kept for
+ * the life of the process, which assumes the device's primary context is never
+ * reset (cudaDeviceReset also invalidates every KV table).  All calls share the
  * array: calls that overlap on the GPU race, so do not run two at once.
- * Allocates no memory.
+ * Arguments are checked exactly as hstu_attn_cached_fwd checks them, before the
+ * scratch size.  Allocates no memory.
  */
 HSTU_API size_t hstu_attn_cached_noalloc_max_scratch(void);
 HSTU_API hstu_status hstu_attn_cached_fwd_noalloc(hstu_kv_table* t, const int64_t* users, int32_t B,

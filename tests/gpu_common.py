@@ -31,18 +31,25 @@ def errors(got, ref):
     return max_abs, rel_l2, max_rel
 
 
+# Rounding a value x to bf16 (round to nearest even) moves it by at most half an
+# ulp, i.e. at most 2^-8 |x| (8 significand bits).
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
 def assert_bf16_close(got, ref, what="", ulp_aware=False):
     """The contract bound: max-abs <= 1e-2 and rel-L2 <= 5e-3.
 
-    ulp_aware: for edge-case inputs whose outputs exceed 1 in magnitude, one bf16
-    ulp of the output (2^-7 |x| at most) is itself above 1e-2, so the elementwise
-    bound becomes 1e-2 + 2^-7 |ref|; rel-L2 stays 5e-3."""
+    ulp_aware: for edge-case inputs whose outputs reach 4 or more in magnitude,
+    the final rounding of the output to bf16 alone (half an ulp, up to 2^-8 |x|)
+    can exceed 1e-2, so the elementwise bound becomes 1e-2 + 2^-8 |ref| against
+    the unrounded fp64 reference; rel-L2 stays 5e-3."""
     max_abs, rel_l2, _ = errors(got, ref)
     got64 = np.asarray(got, dtype=np.float64)
     assert np.all(np.isfinite(got64)), what
     if ulp_aware:
         ref64 = np.asarray(ref, dtype=np.float64)
-        excess = float(np.max(np.abs(got64 - ref64) - (BF16_MAX_ABS + 2.0 ** -7 * np.abs(ref64))))
+        excess = float(np.max(np.abs(got64 - ref64) -
+                              (BF16_MAX_ABS + BF16_HALF_ULP_REL * np.abs(ref64))))
         assert excess <= 0 and rel_l2 <= BF16_REL_L2, \
             f"{what}: max_abs={max_abs:.3e} excess={excess:.3e} rel_l2={rel_l2:.3e}"
     else:

@@ -49,3 +49,60 @@ def test_peaks_fall_back_when_the_measured_file_is_absent(tmp_path, monkeypatch)
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}))
     hbm, tf, tf_sus, src = bench.load_peaks()
     assert (hbm, tf, src) == (6000.0, 1500.0, "measured")
+
+
+def test_launcher_command_starts_one_rank_per_gpu():
+    cmd = bench.launcher_command(4, ["--gpus", "4", "--steps", "3"], port=12345)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "12345"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"] and cmd[-5].endswith("bench.py")
+
+
+def test_world_mismatch_is_refused():
+    import pytest
+    assert bench.check_world(1, {}) == (0, 1, 0)
+    assert bench.check_world(2, {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"}) == (1, 2, 1)
+    with pytest.raises(SystemExit):
+        bench.check_world(8, {"WORLD_SIZE": "1", "RANK": "0"})
+
+
+def _rank_worker(rank, world, port, q):
+    import os
+    import hashlib
+    import torch.distributed as dist
+    import workloads as W
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    r, w, local = bench.check_world(world, os.environ)
+    dist.init_process_group("gloo", rank=r, world_size=w)
+    seeds = bench.rank_seeds(r)
+    c = W.cached_cand(seed=seeds["cached_cand"])
+    digest = hashlib.sha256(c.hist_k[:64].tobytes() + c.q_cand[:64].tobytes()).hexdigest()
+    q.put((r, local, seeds, c.hist_lengths.tolist(), digest))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_get_distinct_user_batches():
+    """Weak scaling: each rank of a 2-rank launch reads its rank from the
+    launcher's environment and draws its own batch of users; rank 0's batch is
+    the reference workload."""
+    import os
+    import torch.multiprocessing as mp
+    import workloads as W
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 31500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_rank_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, l0, s0, h0, d0), (r1, l1, s1, h1, d1) = res
+    assert (r0, l0, r1, l1) == (0, 0, 1, 1)
+    assert s0 != s1 and d0 != d1
+    assert h0 == W.cached_cand().hist_lengths.tolist()

@@ -74,11 +74,70 @@ def test_bf16_tcgen05_pos_rab(lengths):
     assert_bf16_close(got, ref, f"bf16 {lengths[:8]}...", ulp_aware=True)
 
 
+@pytest.mark.parametrize("lengths", [[100, 50, 128, 1], [7]])
+def test_bf16_tcgen05_few_short_users(lengths):
+    """Few users of at most one query tile: fewer items than SMs, and no
+    workspace to split keys into, so every item streams all of its keys."""
+    case = workloads.jagged_case(14, lengths, H=4, d=128, dtype="bf16", n_pos=32, n_time=16)
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, f"short users {lengths}", ulp_aware=True)
+
+
 def test_bf16_tcgen05_pos_time_rab():
     case = workloads.jagged_case(8, [200, 640, 37, 1100], H=4, d=128, dtype="bf16", n_pos=128,
                                  n_time=64)
     got, ref = run_case(case)
     assert_bf16_close(got, ref, "pos+time rab")
+
+
+def _bucket_reach(ts, off, n):
+    """Largest unclamped time bucket over visible pairs (floor(log2(max(dt,0)+1)))."""
+    best = 0
+    for b in range(len(off) - 1):
+        t = ts[off[b]:off[b + 1]]
+        dt = np.maximum(t[:, None] - t[None, :], 0)[np.tril_indices(len(t))]
+        best = max(best, int(np.floor(np.log2(dt.max() + 1))))
+    return best
+
+
+EDGE_TS = [
+    ("increasing", 3 * 86400, 128, 64),   # spans of years: integer time buckets
+    ("unordered", 3, 128, 64),            # equal and decreasing neighbours: max(dt, 0)
+    ("unordered", 300, 4, 4),             # both tables clamp at n - 1
+    ("increasing", 20 * 86400, 4, 4),     # clamps on the integer time path
+]
+
+
+@pytest.mark.parametrize("kind,gap,n_pos,n_time", EDGE_TS)
+def test_bf16_tcgen05_rab_edge_timestamps_and_tables(kind, gap, n_pos, n_time):
+    """Time-gap bias branches that the workloads' Exp(300 s) gaps never reach."""
+    lengths = [700, 129, 1500, 64]
+    case = workloads.jagged_case(12, lengths, H=4, d=128, dtype="bf16", n_pos=n_pos,
+                                 n_time=n_time, ts_gap_mean=gap, ts_kind=kind)
+    ts, off = case.timestamps, case.seq_offsets
+    spans = [int(ts[off[b + 1] - 1] - ts[off[b]]) for b in range(len(lengths))]
+    steps = np.concatenate([np.diff(ts[off[b]:off[b + 1]]) for b in range(len(lengths))])
+    if kind == "increasing" and gap > 86400:
+        assert max(spans) > 2 ** 23            # offsets leave the exact float range
+    if kind == "unordered":
+        assert np.any(steps == 0) and np.any(steps < 0)
+    if n_time == 4:
+        assert _bucket_reach(ts, off, n_time) > n_time - 1   # the time clamp bites
+        assert max(lengths) > 2 ** n_pos                      # so does the position clamp
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, f"{kind} gaps {gap}, tables {n_pos}/{n_time}")
+
+
+@pytest.mark.parametrize("d,dtype", [(32, "f32"), (64, "bf16")])
+@pytest.mark.parametrize("kind,gap", [("increasing", 3 * 86400), ("unordered", 3)])
+def test_simt_rab_edge_timestamps_and_tables(d, dtype, kind, gap):
+    case = workloads.jagged_case(13, [90, 300, 17], H=2, d=d, dtype=dtype, n_pos=4, n_time=4,
+                                 ts_gap_mean=gap, ts_kind=kind)
+    got, ref = run_case(case)
+    if dtype == "f32":
+        assert_f32_close(got, ref, f"simt fp32 {kind}")
+    else:
+        assert_bf16_close(got, ref, f"simt bf16 {kind}")
 
 
 def test_bf16_no_rab_and_single_head():

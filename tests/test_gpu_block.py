@@ -1,9 +1,16 @@
 """hstu_block_fwd (GEMM + SiLU, attention, LayerNorm gate, GEMM + residual) vs the oracle.
 
-Tolerance for bf16 tensors whose magnitude exceeds 1: a rounding flip of one
-bf16 ulp is 2^-7 |x| at |x| in [1, 2) and more above; both sides round X to
-bf16 at the same points, so a value may land one ulp apart.  Hence
-|err| <= 1e-2 + 2^-7 |ref| elementwise, and rel-L2 <= 5e-3 overall.
+The contract is per-layer parity: the oracle layer is fed the GPU's own input
+to that layer and rounds to bf16 where the GPU stores bf16 (UVQK, A, G), but its
+final residual sum X + G W2 is left unrounded.  The GPU's bf16 X' is that sum
+computed in fp32 and rounded once, so |GPU - ref| <= (fp32 and operand-rounding
+error, within 1e-2) + half an ulp of X' (<= 2^-8 |X'|): the elementwise bound is
+1e-2 + 2^-8 |ref|, and rel-L2 <= 5e-3.
+
+The multi-layer chain is reported as a diagnostic: a rounding point whose two
+sides land on adjacent bf16 values at layer l moves every later layer, so no
+elementwise bound follows from the per-layer one.  It is checked only with the
+rel-L2 bound.
 """
 
 import numpy as np
@@ -12,21 +19,28 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import dev, storage, to_np
+from tests.gpu_common import BF16_HALF_ULP_REL, dev, storage, to_np
 
 pytestmark = pytest.mark.gpu
 
-ATOL, RTOL, REL_L2 = 1e-2, 2.0 ** -7, 5e-3
+ATOL, REL_L2 = 1e-2, 5e-3
 
 
 def assert_block_close(got, ref, what):
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     err = np.abs(got - ref)
-    bound = ATOL + RTOL * np.abs(ref)
+    bound = ATOL + BF16_HALF_ULP_REL * np.abs(ref)
     rel_l2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     worst = float(np.max(err - bound))
     assert np.all(np.isfinite(got)) and worst <= 0 and rel_l2 <= REL_L2, \
         f"{what}: worst excess={worst:.3e} max_abs={err.max():.3e} rel_l2={rel_l2:.3e}"
+
+
+def chain_diagnostic(got, ref, what):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    rel_l2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    print(f"{what}: chain max_abs={np.max(np.abs(got - ref)):.3e} rel_l2={rel_l2:.3e}")
+    assert np.all(np.isfinite(got)) and rel_l2 <= REL_L2, f"{what}: rel_l2={rel_l2:.3e}"
 
 
 def gpu_layers(case, x0, layers):
@@ -47,24 +61,26 @@ def gpu_layers(case, x0, layers):
     return outs
 
 
-def oracle_layer(case, x_in, l, rows_of=None):
+def oracle_layer(case, x_in, l):
+    """Layer l on x_in, every bf16 rounding point except the final one."""
     return oracle.hstu_block(x_in, case.seq_offsets, case.w_uvqk[l:l + 1], case.w_o[l:l + 1],
                              case.timestamps, case.pos_table, case.time_table, case.scale,
-                             H=case.H, dh=case.dh, round_bf16=True)
+                             H=case.H, dh=case.dh, round_bf16=True, round_output=False)
+
+
+def check_per_layer(case, outs, layers, what):
+    for l in layers:
+        x_in = case.x0 if l == 0 else outs[l - 1]
+        assert_block_close(outs[l], oracle_layer(case, x_in, l), f"{what}, layer {l}")
 
 
 def test_block_small_per_layer_and_chain():
     case = workloads.block_case(31, [130, 257, 40], n_layers=2)
     outs = gpu_layers(case, case.x0, range(2))
-    # per layer: the oracle layer applied to the GPU's own input
-    x_in = case.x0
-    for l in range(2):
-        ref = oracle_layer(case, x_in, l)
-        assert_block_close(outs[l], ref, f"layer {l}")
-        x_in = outs[l]
+    check_per_layer(case, outs, range(2), "small")
     chain = oracle.hstu_block(case.x0, case.seq_offsets, case.w_uvqk, case.w_o, case.timestamps,
                               case.pos_table, case.time_table, case.scale, H=case.H, dh=case.dh)
-    assert_block_close(outs[-1], chain, "2-layer chain")
+    chain_diagnostic(outs[-1], chain, "2-layer chain")
 
 
 def test_block_all_layers_in_one_call_equals_layer_by_layer():
@@ -79,25 +95,34 @@ def test_block_all_layers_in_one_call_equals_layer_by_layer():
     assert np.array_equal(to_np(x), outs[-1])
 
 
-def test_block_stack_workload_full_size_one_user():
-    """8 layers, 8 users, L~U[512,4096]: users are independent, so the oracle checks the
-    shortest user's rows, layer by layer on the GPU's own inputs, and the 8-layer chain."""
+def test_block_stack_workload_full_size_all_users():
+    """8 layers, 8 users, L~U[512,4096] (T ~ 18k): every row of every user at layers
+    0, 3 and 7 against the oracle layer on the GPU's own input; the 8-layer chain
+    as a diagnostic."""
     case = workloads.block_stack()
     outs = gpu_layers(case, case.x0, range(case.n_layers))
-    b = int(np.argmin(case.lengths))
-    s, e = int(case.seq_offsets[b]), int(case.seq_offsets[b + 1])
-    sub = workloads.BlockCase("one_user", case.lengths[b:b + 1], np.array([0, e - s]), case.d_model,
-                              case.H, case.dh, case.n_layers, case.x0[s:e], case.w_uvqk, case.w_o,
-                              case.pos_table, case.time_table, case.timestamps[s:e], case.scale)
-    x_in = sub.x0
-    for l in (0, 3, 7):
-        x_in = case.x0[s:e] if l == 0 else outs[l - 1][s:e]
-        ref = oracle_layer(sub, x_in, l)
-        assert_block_close(outs[l][s:e], ref, f"full size, layer {l}")
-    # the 8-layer chain: rounding differences compound through the residual stream, so
-    # the elementwise bound is looser (per-layer parity above is the contract)
-    chain = oracle.hstu_block(sub.x0, sub.seq_offsets, sub.w_uvqk, sub.w_o, sub.timestamps,
-                              sub.pos_table, sub.time_table, sub.scale, H=sub.H, dh=sub.dh)
-    got = np.asarray(outs[-1][s:e], np.float64)
-    rel_l2 = np.linalg.norm(got - chain) / np.linalg.norm(chain)
-    assert rel_l2 <= REL_L2 and np.max(np.abs(got - chain)) <= 0.1, rel_l2
+    check_per_layer(case, outs, (0, 3, 7), "full size")
+    chain = oracle.hstu_block(case.x0, case.seq_offsets, case.w_uvqk, case.w_o, case.timestamps,
+                              case.pos_table, case.time_table, case.scale, H=case.H, dh=case.dh)
+    chain_diagnostic(outs[-1], chain, "8-layer chain")
+
+
+@pytest.mark.parametrize("kind,gap,n_pos,n_time", [
+    ("increasing", 3 * 86400, 128, 64),   # spans of years: integer time buckets
+    ("unordered", 3, 128, 64),            # equal and decreasing neighbours: max(dt, 0)
+    ("unordered", 300, 4, 4),             # both tables clamp at n - 1
+    ("increasing", 20 * 86400, 4, 4),     # clamps on the integer time path
+])
+def test_block_rab_edge_timestamps_and_tables(kind, gap, n_pos, n_time):
+    case = workloads.block_case(33, [300, 700, 129], n_layers=1, n_pos=n_pos, n_time=n_time,
+                                ts_gap_mean=gap, ts_kind=kind)
+    outs = gpu_layers(case, case.x0, range(1))
+    check_per_layer(case, outs, range(1), f"{kind} gaps {gap}, tables {n_pos}/{n_time}")
+
+
+def test_block_few_short_users():
+    """Users of at most 128 tokens and fewer items than SMs (no key splits: the
+    block's workspace holds none)."""
+    case = workloads.block_case(34, [100, 60, 128], n_layers=1)
+    outs = gpu_layers(case, case.x0, range(1))
+    check_per_layer(case, outs, range(1), "few short users")

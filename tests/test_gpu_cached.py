@@ -10,10 +10,6 @@ from tests.gpu_common import assert_bf16_close, assert_f32_close, dev, sample_ro
 
 pytestmark = pytest.mark.gpu
 
-# Causal launches with 256+ query rows can run on single CTAs or on CTA pairs
-# (HSTU_ATTN_CTA_PAIRS forces the choice); the causal tests cover both.
-CTA_PAIRS = pytest.mark.parametrize("cta_pairs", ["0", "1"])
-
 
 def prefill(table, case, users_t):
     """Alloc + append the pre-filled history (untimed set-up of every cached workload)."""
@@ -136,10 +132,8 @@ def test_candidates_workload_full_size():
     table.close()
 
 
-@CTA_PAIRS
 @pytest.mark.parametrize("lengths", [[64, 300, 1000], [17, 64, 129]])
-def test_causal_suffix_small(lengths, cta_pairs, monkeypatch):
-    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
+def test_causal_suffix_small(lengths):
     case = workloads.long_history(lengths=lengths, pool_tokens=4096)
     table = make_table(case)
     users = dev(case.users)
@@ -165,12 +159,10 @@ def test_causal_suffix_decode_queries_only():
     table.close()
 
 
-@CTA_PAIRS
 @pytest.mark.parametrize("lengths", [[255, 256, 257, 384, 385, 1], [1000, 130, 640]])
-def test_causal_suffix_query_blocks(lengths, cta_pairs, monkeypatch):
-    """Runs of 256+ queries go to CTA pairs (256-row blocks, one 128-row half per
-    CTA): block boundaries, a half with no valid rows, a lone row."""
-    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
+def test_causal_suffix_query_blocks(lengths):
+    """Several 128-row query tiles per user: tile boundaries, a ragged last tile,
+    a lone row."""
     case = workloads.long_history(lengths=lengths, pool_tokens=8192)
     table = make_table(case)
     users = dev(case.users)
@@ -180,12 +172,10 @@ def test_causal_suffix_query_blocks(lengths, cta_pairs, monkeypatch):
     table.close()
 
 
-@CTA_PAIRS
-def test_causal_suffix_long_runs_behind_history(cta_pairs, monkeypatch):
-    """Query suffixes of 256-700 rows after long cached histories (block rows start
+def test_causal_suffix_long_runs_behind_history():
+    """Query suffixes of 256-700 rows after long cached histories (tile rows start
     past position 0)."""
     import dataclasses
-    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
     case = workloads.long_history(lengths=[2000, 300, 3000], pool_tokens=8192)
     nq = np.array([300, 256, 700], dtype=np.int64)
     qo = workloads.offsets_from_lengths(case.total_lengths)
@@ -199,10 +189,8 @@ def test_causal_suffix_long_runs_behind_history(cta_pairs, monkeypatch):
     table.close()
 
 
-@CTA_PAIRS
-def test_long_history_workload_full_size_sampled(cta_pairs, monkeypatch):
+def test_long_history_workload_full_size_sampled():
     """32 users, Zipf lengths in [64,16384], 2M-token pool; oracle on sampled rows."""
-    monkeypatch.setenv("HSTU_ATTN_CTA_PAIRS", cta_pairs)
     case = workloads.long_history()
     table = make_table(case)
     users = dev(case.users)
@@ -349,4 +337,32 @@ def test_causal_suffix_short_runs_split_over_keys():
     prefill(table, case, users)
     out = step(table, case, users)
     assert_bf16_close(to_np(out), oracle_out(case), "short causal runs", ulp_aware=True)
+    table.close()
+
+
+def many_user_case(B=1025, n_cand=4, seed=41):
+    """B users with short histories (1..399 tokens, the last one the longest) and a
+    few candidates each: more users than one launch of the tcgen05 kernel takes."""
+    rng = np.random.default_rng(seed)
+    hist = rng.integers(1, 400, size=B)
+    hist[-1] = 399
+    base = workloads.cached_cand(B=2, hmin=0, hmax=1, n_new=0, n_cand=n_cand, seed=seed)
+    return _with_lengths(base, hist, 0, n_cand, seed=seed + 1)
+
+
+def test_candidates_over_1024_users_split_remainder_chunk():
+    """1025 users run as a chunk of 1024 (no key split: its items already fill the
+    GPU) and a chunk of one user whose keys are split over several CTAs.  The
+    workspace query must cover the last chunk's partials, and that chunk's reduce
+    must leave the first chunk's finished rows alone."""
+    import generative_recommender_sequence_b200 as hstu
+    case = many_user_case()
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    total_q, max_cached = int(case.q_offsets[-1]), int(case.total_lengths.max())
+    need = table.workspace_size(case.B, total_q, 4, max_cached, hstu.HSTU_MASK_CANDIDATES)
+    assert need > 0
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), "1025 users", ulp_aware=True)
     table.close()

@@ -69,3 +69,52 @@ def test_lru_eviction_offload_and_onboard_round_trip():
                                  pos_table=pt, scale=1.0 / (L + nc))
     assert_bf16_close(to_np(out), ref, "onboarded user", ulp_aware=True)
     table.close()
+
+
+def test_multi_layer_eviction_and_onboarding_with_the_cached_block_step():
+    """Per-layer caches of the cached block step under a pool that is too small:
+    a user evicted from every layer (K/V offloaded to host memory) and brought
+    back later gives, bit for bit, the results of the same requests served
+    with a pool large enough that nothing is evicted."""
+    import generative_recommender_sequence_b200 as hstu
+    from generative_recommender_sequence_b200.kv_cache import KVCacheManager
+    rng = np.random.default_rng(23)
+    DM, L = 512, 2
+    bf = lambda a: workloads._as_storage(np.asarray(a, np.float32), "bf16")
+    w1 = [storage(bf(rng.normal(0, 0.02, (DM, 4 * DM))), "bf16") for _ in range(L)]
+    w2 = [storage(bf(rng.normal(0, 0.02, (DM, DM))), "bf16") for _ in range(L)]
+    pt = dev(rng.normal(0, 0.1, 16).astype(np.float32))
+    requests = [([0, 1], [100, 150], 0), ([2], [40], 0), ([0], [10], 8)]
+    xs = [(bf(rng.standard_normal((sum(n), DM))), bf(rng.standard_normal((len(u) * c, DM))))
+          for u, n, c in requests]
+    scale = 1.0 / 200
+
+    def serve_all(n_pages):
+        tables = [hstu.KVTable(n_pages, H, D, max_users=4, max_pages_per_user=16,
+                               free_order=np.random.default_rng(3 + l).permutation(n_pages))
+                  for l in range(L)]
+        mgr = KVCacheManager(tables)
+        outs = []
+        for (users, n_new, n_c), (x_new, x_c) in zip(requests, xs):
+            mgr.make_room(users, n_new)
+            x = storage(np.concatenate([x_new, x_c]), "bf16")
+            off = lambda n: dev(workloads.offsets_from_lengths(np.array(n)))
+            max_cached = max(mgr.cached_length(u) + n for u, n in zip(users, n_new))
+            hstu.block_cached_step(tables, dev(np.array(users, np.int64)), x, off(n_new), max(n_new),
+                                   off([n_c] * len(users)) if n_c else None, n_c, max_cached, w1, w2,
+                                   pos_table=pt, scale=scale, T_new=int(sum(n_new)))
+            mgr.commit(users, n_new)
+            outs.append(to_np(x))
+        torch.cuda.synchronize()
+        for t in tables:
+            assert t.status() == 0
+            t.close()
+        return mgr, outs
+
+    small, got = serve_all(10)
+    assert small.evicted == [0, 1] and small.onboarded == [0]
+    big, ref = serve_all(64)
+    assert big.evicted == []
+    for g, r in zip(got, ref):
+        assert np.array_equal(g, r)
+    assert hstu.last_device_error() == 0

@@ -68,11 +68,23 @@ def offsets_from_lengths(lengths) -> np.ndarray:
     return off
 
 
-def draw_timestamps(rng: np.random.Generator, lengths) -> np.ndarray:
-    """Strictly increasing int64 timestamps per user: TS0, then gaps 1+floor(Exp(300))."""
+def draw_timestamps(rng: np.random.Generator, lengths, gap_mean: float = GAP_MEAN_S,
+                    kind: str = "increasing") -> np.ndarray:
+    """int64 timestamps per user, starting at TS0.
+
+    kind "increasing": gaps 1 + floor(Exp(gap_mean)), strictly increasing (the
+    workloads' recipe; gap_mean of days gives spans of years).
+    kind "unordered": gaps uniform in [-gap_mean, gap_mean], so neighbours may be
+    equal or decreasing (logs merged from several sources)."""
+    if kind not in ("increasing", "unordered"):
+        raise ValueError(kind)
     out = []
     for L in lengths:
-        gaps = 1 + np.floor(rng.exponential(GAP_MEAN_S, size=int(L) - 1)).astype(np.int64)
+        if kind == "increasing":
+            gaps = 1 + np.floor(rng.exponential(gap_mean, size=int(L) - 1)).astype(np.int64)
+        else:
+            g = int(gap_mean)
+            gaps = rng.integers(-g, g, size=int(L) - 1, endpoint=True).astype(np.int64)
         ts = np.empty(int(L), dtype=np.int64)
         ts[0] = TS0
         if L > 1:
@@ -118,13 +130,14 @@ class JaggedCase:
 
 def jagged_case(seed: int, lengths, H: int, d: int, dtype: str = "bf16",
                 n_pos: int = 16, n_time: int = 0, scale: Optional[float] = None,
-                name: str = "custom", rng: Optional[np.random.Generator] = None) -> JaggedCase:
+                name: str = "custom", rng: Optional[np.random.Generator] = None,
+                ts_gap_mean: float = GAP_MEAN_S, ts_kind: str = "increasing") -> JaggedCase:
     """Build a jagged causal case with given lengths (rab tables ~ N(0, 0.1))."""
     rng = rng if rng is not None else np.random.default_rng(seed)
     lengths = np.asarray(lengths, dtype=np.int64)
     off = offsets_from_lengths(lengths)
     T = int(off[-1])
-    ts = draw_timestamps(rng, lengths) if n_time > 0 else None
+    ts = draw_timestamps(rng, lengths, ts_gap_mean, ts_kind) if n_time > 0 else None
     pos_table = rng.normal(0.0, 0.1, size=n_pos).astype(np.float32)
     time_table = rng.normal(0.0, 0.1, size=n_time).astype(np.float32) if n_time > 0 else None
     q = _as_storage(rng.standard_normal((T, H, d), dtype=np.float32), dtype)
@@ -304,14 +317,16 @@ class BlockCase:
 
 
 def block_case(seed: int, lengths, n_layers: int, d_model: int = 512, H: int = 4, dh: int = 128,
-               rng: Optional[np.random.Generator] = None, name: str = "custom") -> BlockCase:
+               rng: Optional[np.random.Generator] = None, name: str = "custom",
+               n_pos: int = 128, n_time: int = 64, ts_gap_mean: float = GAP_MEAN_S,
+               ts_kind: str = "increasing") -> BlockCase:
     rng = rng if rng is not None else np.random.default_rng(seed)
     lengths = np.asarray(lengths, dtype=np.int64)
     off = offsets_from_lengths(lengths)
     T = int(off[-1])
-    ts = draw_timestamps(rng, lengths)
-    pos_table = rng.normal(0.0, 0.1, size=128).astype(np.float32)
-    time_table = rng.normal(0.0, 0.1, size=64).astype(np.float32)
+    ts = draw_timestamps(rng, lengths, ts_gap_mean, ts_kind)
+    pos_table = rng.normal(0.0, 0.1, size=n_pos).astype(np.float32)
+    time_table = rng.normal(0.0, 0.1, size=n_time).astype(np.float32)
     x0 = _as_storage(rng.standard_normal((T, d_model), dtype=np.float32), "bf16")
     w1 = _as_storage(rng.normal(0.0, 0.02, size=(n_layers, d_model, 4 * H * dh)).astype(np.float32), "bf16")
     w2 = _as_storage(rng.normal(0.0, 0.02, size=(n_layers, H * dh, d_model)).astype(np.float32), "bf16")
