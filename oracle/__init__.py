@@ -66,6 +66,10 @@ def _load():
             lib.oracle_attn_causal.restype = I
             lib.oracle_attn_candidates.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, I, D, P, L, P, I]
             lib.oracle_attn_candidates.restype = I
+            lib.oracle_attn_causal_magnitude.argtypes = lib.oracle_attn_causal.argtypes + [I]
+            lib.oracle_attn_causal_magnitude.restype = I
+            lib.oracle_attn_candidates_magnitude.argtypes = lib.oracle_attn_candidates.argtypes + [I]
+            lib.oracle_attn_candidates_magnitude.restype = I
             lib.oracle_layernorm_gate.argtypes = [L, L, P, P, D, I, P, I]
             lib.oracle_layernorm_gate.restype = I
             lib.oracle_hstu_block.argtypes = [L, I, P, I, I, I, I, P, P, P, P, P, I, P, I, D, D, I, I, P, I]
@@ -90,6 +94,9 @@ def _p(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+_MAGNITUDE_KIND = {"silu": 1, "score": 2}
+
+
 def pos_bucket(delta: int, n_buckets: int) -> int:
     return _load().oracle_pos_bucket(int(delta), int(n_buckets))
 
@@ -109,10 +116,14 @@ def round_bf16(x) -> np.ndarray:
 
 
 def attn_causal(q, k, v, kv_offsets, q_offsets=None, timestamps=None, pos_table=None,
-                time_table=None, scale=1.0, rows=None, threads=None) -> np.ndarray:
+                time_table=None, scale=1.0, rows=None, threads=None,
+                magnitude=None) -> np.ndarray:
     """Causal HSTU attention; the queries of user b are its last nq_b tokens.
 
     q: [Tq,H,dqk], k: [Tk,H,dqk], v: [Tk,H,dv]; returns fp64 [Tq or len(rows), H, dv].
+    magnitude="silu" returns |scale| * sum_j |SiLU(s_j)| |v_j| and magnitude="score"
+    |scale| * sum_j |s_j| |v_j| (s_j = q . k_j + rab) instead: the sizes of the
+    sum's terms, for rounding-error bounds, not attention results.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     kv_off = _i64(kv_offsets)
@@ -125,18 +136,24 @@ def attn_causal(q, k, v, kv_offsets, q_offsets=None, timestamps=None, pos_table=
     rows_a = _i64(rows)
     n_rows = len(rows_a) if rows_a is not None else int(q_off[-1])
     out = np.zeros((n_rows, H, dv), dtype=np.float64)
-    rc = _load().oracle_attn_causal(B, H, dqk, dv, _p(kv_off), _p(q_off), _p(q), _p(k), _p(v),
-                                    _p(ts), _p(pt), 0 if pt is None else len(pt), _p(tt),
-                                    0 if tt is None else len(tt), float(scale), _p(rows_a),
-                                    n_rows, _p(out), threads or default_threads())
+    args = (B, H, dqk, dv, _p(kv_off), _p(q_off), _p(q), _p(k), _p(v), _p(ts), _p(pt),
+            0 if pt is None else len(pt), _p(tt), 0 if tt is None else len(tt), float(scale),
+            _p(rows_a), n_rows, _p(out), threads or default_threads())
+    if magnitude is None:
+        rc = _load().oracle_attn_causal(*args)
+    else:
+        rc = _load().oracle_attn_causal_magnitude(*args, _MAGNITUDE_KIND[magnitude])
     if rc != 0:
         raise ValueError("oracle_attn_causal: bad arguments")
     return out
 
 
 def attn_candidates(hist_k, hist_v, hist_offsets, q, k_cand, v_cand, cand_offsets,
-                    pos_table=None, scale=1.0, rows=None, threads=None) -> np.ndarray:
-    """Candidates of user b attend to all of b's cached tokens plus themselves."""
+                    pos_table=None, scale=1.0, rows=None, threads=None,
+                    magnitude=None) -> np.ndarray:
+    """Candidates of user b attend to all of b's cached tokens plus themselves.
+
+    magnitude="silu" / "score": term-by-term magnitudes instead (see attn_causal)."""
     hk, hv = _f64(hist_k), _f64(hist_v)
     q, kc, vc = _f64(q), _f64(k_cand), _f64(v_cand)
     ho, co = _i64(hist_offsets), _i64(cand_offsets)
@@ -146,10 +163,13 @@ def attn_candidates(hist_k, hist_v, hist_offsets, q, k_cand, v_cand, cand_offset
     rows_a = _i64(rows)
     n_rows = len(rows_a) if rows_a is not None else int(co[-1])
     out = np.zeros((n_rows, H, dv), dtype=np.float64)
-    rc = _load().oracle_attn_candidates(B, H, dqk, dv, _p(ho), _p(hk), _p(hv), _p(co), _p(q),
-                                        _p(kc), _p(vc), _p(pt), 0 if pt is None else len(pt),
-                                        float(scale), _p(rows_a), n_rows, _p(out),
-                                        threads or default_threads())
+    args = (B, H, dqk, dv, _p(ho), _p(hk), _p(hv), _p(co), _p(q), _p(kc), _p(vc), _p(pt),
+            0 if pt is None else len(pt), float(scale), _p(rows_a), n_rows, _p(out),
+            threads or default_threads())
+    if magnitude is None:
+        rc = _load().oracle_attn_candidates(*args)
+    else:
+        rc = _load().oracle_attn_candidates_magnitude(*args, _MAGNITUDE_KIND[magnitude])
     if rc != 0:
         raise ValueError("oracle_attn_candidates: bad arguments")
     return out

@@ -31,7 +31,8 @@ def ancestry(beam_parent, beam_offsets, b, j, step):
 
 
 def attn_beam_decode(ctx_k, ctx_v, ctx_offsets, q, beam_offsets, step, beam_k, beam_v, beam_parent,
-                     pos_table=None, scale=1.0, threads=None):
+                     pos_table=None, scale=1.0, threads=None, magnitude=None):
+    """Beam outputs of step `step`; magnitude as for ``oracle.attn_causal``."""
     ck, cv = np.asarray(ctx_k, np.float64), np.asarray(ctx_v, np.float64)
     bk, bv = np.asarray(beam_k, np.float64), np.asarray(beam_v, np.float64)
     co, bo = np.asarray(ctx_offsets, np.int64), np.asarray(beam_offsets, np.int64)
@@ -47,4 +48,5 @@ def attn_beam_decode(ctx_k, ctx_v, ctx_offsets, q, beam_offsets, step, beam_k, b
     kv_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
     q_off = np.arange(len(lens) + 1, dtype=np.int64)
     return attn_causal(np.asarray(q, np.float64), np.concatenate(ks), np.concatenate(vs), kv_off,
-                       q_offsets=q_off, pos_table=pos_table, scale=scale, threads=threads)
+                       q_offsets=q_off, pos_table=pos_table, scale=scale, threads=threads,
+                       magnitude=magnitude)

@@ -35,8 +35,13 @@ def user_scores(q, k, pos_q, pos_k, ts_q, ts_k, pos_table, time_table):
     return s
 
 
-def causal(q, k, v, offsets, timestamps=None, pos_table=None, time_table=None, scale=1.0):
+def causal(q, k, v, offsets, timestamps=None, pos_table=None, time_table=None, scale=1.0,
+           magnitude=None):
+    """magnitude "silu" / "score": |scale| * sum of |SiLU(s)| |v| / |s| |v| over the
+    visible keys."""
     q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+    if magnitude:
+        v, scale = np.abs(v), abs(scale)
     out = np.zeros((q.shape[0], q.shape[1], v.shape[2]))
     for b in range(len(offsets) - 1):
         s0, e0 = int(offsets[b]), int(offsets[b + 1])
@@ -46,14 +51,18 @@ def causal(q, k, v, offsets, timestamps=None, pos_table=None, time_table=None, s
         S = user_scores(q[s0:e0], k[s0:e0], pos, pos, ts, ts, pos_table,
                         time_table if ts is not None else None)
         mask = pos[None, :] <= pos[:, None]
-        W = np.where(mask[None], S * _logistic(S), 0.0)
+        W = np.where(mask[None], S if magnitude == "score" else S * _logistic(S), 0.0)
+        if magnitude:
+            W = np.abs(W)
         out[s0:e0] = np.einsum("hij,jhe->ihe", W, v[s0:e0]) * scale
     return out
 
 
 def candidates(hist_k, hist_v, hist_offsets, q, k_cand, v_cand, cand_offsets, pos_table=None,
-               scale=1.0):
+               scale=1.0, magnitude=None):
     hk, hv, q, kc, vc = (np.asarray(x, np.float64) for x in (hist_k, hist_v, q, k_cand, v_cand))
+    if magnitude:
+        hv, vc, scale = np.abs(hv), np.abs(vc), abs(scale)
     out = np.zeros((q.shape[0], q.shape[1], vc.shape[2]))
     for b in range(len(cand_offsets) - 1):
         hs, he = int(hist_offsets[b]), int(hist_offsets[b + 1])
@@ -67,6 +76,8 @@ def candidates(hist_k, hist_v, hist_offsets, q, k_cand, v_cand, cand_offsets, po
         mask = np.zeros((nc, nh + nc), bool)
         mask[:, :nh] = True
         mask[np.arange(nc), nh + np.arange(nc)] = True
-        W = np.where(mask[None], S * _logistic(S), 0.0)
+        W = np.where(mask[None], S if magnitude == "score" else S * _logistic(S), 0.0)
+        if magnitude:
+            W = np.abs(W)
         out[cs:ce] = np.einsum("hij,jhe->ihe", W, vals) * scale
     return out

@@ -151,6 +151,7 @@ typedef struct {
     int64_t n_rows;
     double* out;
     int64_t out_stride; /* elements between consecutive output rows */
+    int magnitude;      /* 0: SiLU(s) * v; 1: |SiLU(s)| * |v|; 2: |s| * |v| */
 } causal_ctx;
 
 static void causal_task(void* vctx, int64_t t) {
@@ -176,10 +177,13 @@ static void causal_task(void* vctx, int64_t t) {
             int64_t ti = c->ts[c->kv_off[b] + pi];
             s += c->time_table[oracle_time_bucket(ti - c->ts[j], c->n_time)];
         }
-        double w = oracle_silu(s);
-        for (int e = 0; e < c->dv; e++) o[e] += w * vj[e];
+        double w = c->magnitude == 2 ? fabs(s) : oracle_silu(s);
+        if (c->magnitude)
+            for (int e = 0; e < c->dv; e++) o[e] += fabs(w) * fabs(vj[e]);
+        else
+            for (int e = 0; e < c->dv; e++) o[e] += w * vj[e];
     }
-    for (int e = 0; e < c->dv; e++) o[e] *= c->scale;
+    for (int e = 0; e < c->dv; e++) o[e] *= c->magnitude ? fabs(c->scale) : c->scale;
 }
 
 /*
@@ -190,11 +194,12 @@ static void causal_task(void* vctx, int64_t t) {
  * rows: query rows to compute (NULL: all Tq rows, in order).
  * Returns 0, or -1 on an argument error.
  */
-int oracle_attn_causal(int B, int H, int dqk, int dv, const int64_t* kv_offsets,
-                       const int64_t* q_offsets, const double* q, const double* k,
-                       const double* v, const int64_t* timestamps, const double* pos_table,
-                       int n_pos, const double* time_table, int n_time, double scale,
-                       const int64_t* rows, int64_t n_rows, double* out, int n_threads) {
+static int attn_causal_impl(int B, int H, int dqk, int dv, const int64_t* kv_offsets,
+                            const int64_t* q_offsets, const double* q, const double* k,
+                            const double* v, const int64_t* timestamps, const double* pos_table,
+                            int n_pos, const double* time_table, int n_time, double scale,
+                            const int64_t* rows, int64_t n_rows, double* out, int n_threads,
+                            int magnitude) {
     if (B < 0 || H <= 0 || dqk <= 0 || dv <= 0) return -1;
     for (int b = 0; b < B; b++) {
         int64_t nk = kv_offsets[b + 1] - kv_offsets[b];
@@ -205,9 +210,36 @@ int oracle_attn_causal(int B, int H, int dqk, int dv, const int64_t* kv_offsets,
     causal_ctx c = {B, H, dqk, dv, kv_offsets, q_offsets, q, k, v,
                     (int64_t)H * dqk, (int64_t)H * dqk, (int64_t)H * dv,
                     timestamps, pos_table, n_pos, time_table, n_time, scale,
-                    rows, rows ? n_rows : q_offsets[B], out, (int64_t)H * dv};
+                    rows, rows ? n_rows : q_offsets[B], out, (int64_t)H * dv, magnitude};
     run_tasks(causal_task, &c, c.n_rows * H, n_threads);
     return 0;
+}
+
+int oracle_attn_causal(int B, int H, int dqk, int dv, const int64_t* kv_offsets,
+                       const int64_t* q_offsets, const double* q, const double* k,
+                       const double* v, const int64_t* timestamps, const double* pos_table,
+                       int n_pos, const double* time_table, int n_time, double scale,
+                       const int64_t* rows, int64_t n_rows, double* out, int n_threads) {
+    return attn_causal_impl(B, H, dqk, dv, kv_offsets, q_offsets, q, k, v, timestamps, pos_table,
+                            n_pos, time_table, n_time, scale, rows, n_rows, out, n_threads, 0);
+}
+
+/*
+ * Magnitudes of the same sum, term by term as above, with s = q_i . k_j + rab(i,j):
+ *   kind 1: |scale| * sum_j |SiLU(s)| * |v_j|
+ *   kind 2: |scale| * sum_j |s| * |v_j|
+ * Not attention results: they size rounding-error bounds (an error relative to
+ * every SiLU term, or proportional to every score, is bounded by these).
+ */
+int oracle_attn_causal_magnitude(int B, int H, int dqk, int dv, const int64_t* kv_offsets,
+                                 const int64_t* q_offsets, const double* q, const double* k,
+                                 const double* v, const int64_t* timestamps,
+                                 const double* pos_table, int n_pos, const double* time_table,
+                                 int n_time, double scale, const int64_t* rows, int64_t n_rows,
+                                 double* out, int n_threads, int kind) {
+    if (kind != 1 && kind != 2) return -1;
+    return attn_causal_impl(B, H, dqk, dv, kv_offsets, q_offsets, q, k, v, timestamps, pos_table,
+                            n_pos, time_table, n_time, scale, rows, n_rows, out, n_threads, kind);
 }
 
 /* ------------------------------------------------------------------ */
@@ -224,6 +256,7 @@ typedef struct {
     const int64_t* rows;
     int64_t n_rows;
     double* out;
+    int magnitude; /* 0: SiLU(s) * v; 1: |SiLU(s)| * |v|; 2: |s| * |v| */
 } cand_ctx;
 
 static void cand_task(void* vctx, int64_t t) {
@@ -250,10 +283,13 @@ static void cand_task(void* vctx, int64_t t) {
         double s = 0.0;
         for (int e = 0; e < c->dqk; e++) s += qc[e] * kj[e];
         if (c->pos_table) s += c->pos_table[oracle_pos_bucket(pc - (pj < nh ? pj : pc), c->n_pos)];
-        double w = oracle_silu(s);
-        for (int e = 0; e < c->dv; e++) o[e] += w * vj[e];
+        double w = c->magnitude == 2 ? fabs(s) : oracle_silu(s);
+        if (c->magnitude)
+            for (int e = 0; e < c->dv; e++) o[e] += fabs(w) * fabs(vj[e]);
+        else
+            for (int e = 0; e < c->dv; e++) o[e] += w * vj[e];
     }
-    for (int e = 0; e < c->dv; e++) o[e] *= c->scale;
+    for (int e = 0; e < c->dv; e++) o[e] *= c->magnitude ? fabs(c->scale) : c->scale;
 }
 
 /*
@@ -268,7 +304,23 @@ int oracle_attn_candidates(int B, int H, int dqk, int dv, const int64_t* hist_of
                            const int64_t* rows, int64_t n_rows, double* out, int n_threads) {
     if (B < 0 || H <= 0 || dqk <= 0 || dv <= 0) return -1;
     cand_ctx c = {B, H, dqk, dv, hist_offsets, cand_offsets, hist_k, hist_v, q, k_cand,
-                  v_cand, pos_table, n_pos, scale, rows, rows ? n_rows : cand_offsets[B], out};
+                  v_cand, pos_table, n_pos, scale, rows, rows ? n_rows : cand_offsets[B], out, 0};
+    run_tasks(cand_task, &c, c.n_rows * H, n_threads);
+    return 0;
+}
+
+/* Magnitudes of the candidate sum, term by term (kinds as for
+ * oracle_attn_causal_magnitude). */
+int oracle_attn_candidates_magnitude(int B, int H, int dqk, int dv, const int64_t* hist_offsets,
+                                     const double* hist_k, const double* hist_v,
+                                     const int64_t* cand_offsets, const double* q,
+                                     const double* k_cand, const double* v_cand,
+                                     const double* pos_table, int n_pos, double scale,
+                                     const int64_t* rows, int64_t n_rows, double* out,
+                                     int n_threads, int kind) {
+    if (B < 0 || H <= 0 || dqk <= 0 || dv <= 0 || (kind != 1 && kind != 2)) return -1;
+    cand_ctx c = {B, H, dqk, dv, hist_offsets, cand_offsets, hist_k, hist_v, q, k_cand,
+                  v_cand, pos_table, n_pos, scale, rows, rows ? n_rows : cand_offsets[B], out, kind};
     run_tasks(cand_task, &c, c.n_rows * H, n_threads);
     return 0;
 }

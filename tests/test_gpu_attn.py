@@ -6,8 +6,8 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import (assert_bf16_close, assert_f32_close, dev, sample_rows, storage,
-                              to_np)
+from tests.gpu_common import (assert_bf16_close, assert_f32_close, dev, magnitudes, sample_rows,
+                              storage, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -18,6 +18,12 @@ def _gpu():
     if not torch.cuda.is_available():
         pytest.fail("a CUDA device is required for -m gpu tests")
     hstu.device_check()
+
+
+def case_magnitudes(case, rows=None):
+    return magnitudes(oracle.attn_causal, case.q, case.k, case.v, case.seq_offsets,
+                      timestamps=case.timestamps, pos_table=case.pos_table,
+                      time_table=case.time_table, scale=case.scale, rows=rows)
 
 
 def run_case(case, rows=None, stream=None):
@@ -71,7 +77,7 @@ def test_bf16_tcgen05_pos_rab(lengths):
     # units and one bf16 ulp exceeds 1e-2 -> the ulp-aware elementwise bound
     case = workloads.jagged_case(7, lengths, H=4, d=128, dtype="bf16", n_pos=16)
     got, ref = run_case(case)
-    assert_bf16_close(got, ref, f"bf16 {lengths[:8]}...", ulp_aware=True)
+    assert_bf16_close(got, ref, f"bf16 {lengths[:8]}...", mag=case_magnitudes(case))
 
 
 @pytest.mark.parametrize("lengths", [[100, 50, 128, 1], [7]])
@@ -80,7 +86,7 @@ def test_bf16_tcgen05_few_short_users(lengths):
     workspace to split keys into, so every item streams all of its keys."""
     case = workloads.jagged_case(14, lengths, H=4, d=128, dtype="bf16", n_pos=32, n_time=16)
     got, ref = run_case(case)
-    assert_bf16_close(got, ref, f"short users {lengths}", ulp_aware=True)
+    assert_bf16_close(got, ref, f"short users {lengths}", mag=case_magnitudes(case))
 
 
 def test_bf16_tcgen05_pos_time_rab():

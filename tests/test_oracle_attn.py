@@ -235,3 +235,44 @@ def test_sampled_candidate_rows():
     full = oracle.attn_candidates(**a)
     rows = np.array([5, 1])
     assert np.array_equal(oracle.attn_candidates(**a, rows=rows), full[rows])
+
+
+# ------------------------------------------------------------------ magnitude sums
+# |scale| * sum_j |SiLU(q.k_j + rab)| * |v_j| sizes the error bound of a GPU path
+# whose per-term error is relative (bf16 P operand); it is pinned like the sum.
+
+@pytest.mark.parametrize("kind", ["silu", "score"])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_magnitude_matches_brute_force_twin(seed, kind):
+    rng = np.random.default_rng(300 + seed)
+    lengths = rng.integers(1, 30, size=3)
+    case = jagged_case(seed, lengths, H=2, d=5, dtype="f32", n_pos=9, n_time=7)
+    args = dict(timestamps=case.timestamps, pos_table=case.pos_table, time_table=case.time_table,
+                scale=-case.scale)
+    got = oracle.attn_causal(case.q, case.k, case.v, case.seq_offsets, magnitude=kind, **args)
+    ref = brute.causal(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                       case.pos_table, case.time_table, -case.scale, magnitude=kind)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    a = _cand_case(310 + seed, [0, 5, 23], [2, 1, 5], d=3, n_pos=6)
+    np.testing.assert_allclose(oracle.attn_candidates(**a, magnitude=kind),
+                               brute.candidates(**a, magnitude=kind), rtol=1e-12, atol=1e-12)
+
+
+def test_magnitude_bounds_the_sum_and_equals_it_for_nonnegative_terms():
+    case = jagged_case(21, [13, 40], H=2, d=4, dtype="f32", n_pos=16)
+    f = lambda v, mag, rab: oracle.attn_causal(case.q, case.k, v, case.seq_offsets,
+                                               pos_table=np.full(16, rab), scale=case.scale,
+                                               magnitude=mag)
+    # triangle inequality, term by term; |SiLU(s)| <= |s| for every s
+    assert np.all(f(case.v, "silu", 0.1) >= np.abs(f(case.v, None, 0.1)))
+    assert np.all(f(case.v, "score", 0.1) >= f(case.v, "silu", 0.1))
+    # rab = 60 keeps every SiLU argument positive (|q.k| < 60 here) and |v| >= 0:
+    # every term is non-negative, so the magnitude is the sum itself, bit for bit
+    s = np.einsum("ihe,jhe->ihj", case.q.astype(np.float64), case.k.astype(np.float64))
+    assert np.max(np.abs(s)) < 60
+    v_pos = np.abs(case.v)
+    assert np.array_equal(f(v_pos, "silu", 60.0), f(v_pos, None, 60.0))
+    a = _cand_case(22, [7, 3], [2, 4])
+    a["hist_v"], a["v_cand"] = np.abs(a["hist_v"]), np.abs(a["v_cand"])
+    a["pos_table"] = np.full(16, 60.0)
+    assert np.array_equal(oracle.attn_candidates(**a, magnitude="silu"), oracle.attn_candidates(**a))

@@ -18,12 +18,12 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import assert_bf16_close, dev, storage, to_np
+from tests.gpu_common import assert_bf16_close, dev, magnitudes, storage, to_np
 
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_candidates(case):
+def _oracle_candidates(case, magnitude=None):
     ho = workloads.offsets_from_lengths(case.hist_lengths)
     no = workloads.offsets_from_lengths(case.n_new)
     ks, vs = [], []
@@ -33,7 +33,7 @@ def _oracle_candidates(case):
     return oracle.attn_candidates(np.concatenate(ks), np.concatenate(vs),
                                   workloads.offsets_from_lengths(case.total_lengths), case.q_cand,
                                   case.k_cand, case.v_cand, case.q_offsets,
-                                  pos_table=case.pos_table, scale=case.scale)
+                                  pos_table=case.pos_table, scale=case.scale, magnitude=magnitude)
 
 
 def _noalloc(lib, table, users, case, q, kc, vc, q_off, max_q, max_cached, rab, out, mask=0):
@@ -118,7 +118,8 @@ def test_noalloc_over_1024_users():
     torch.cuda.synchronize()
     assert table.status() == 0 and hstu.last_device_error() == 0
     assert torch.equal(out, ref)
-    assert_bf16_close(to_np(out), _oracle_candidates(case), "noalloc, 1025 users", ulp_aware=True)
+    assert_bf16_close(to_np(out), _oracle_candidates(case), "noalloc, 1025 users",
+                      mag=magnitudes(lambda **kw: _oracle_candidates(case, **kw)))
     table.close()
 
 
