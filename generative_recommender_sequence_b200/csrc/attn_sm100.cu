@@ -125,10 +125,10 @@ struct __align__(1024) Smem {
 
 struct KParams {
   int B, H, mode, n_split, kps;
-  // balanced key splits: per-user split counts chosen on the device, one item
-  // per CTA; partial sums of item t at partial + t * BM * HD, and the item
-  // offsets per user (int32 [B + 1]) written to plan for the reduce
-  int balanced;
+  // balanced key splits (the BAL kernels): per-user split counts chosen on
+  // the device, one item per CTA; partial sums of item t at
+  // partial + t * BM * HD, and the item offsets per user (int32 [B + 1])
+  // written to plan for the reduce
   int* plan;
   const int64_t* q_off;
   const int64_t* kv_off;
@@ -239,7 +239,7 @@ struct Item {
 };
 
 // Item m of user b covers query rows [BM m, BM m + BM).
-template <bool PAGED, bool CAND>
+template <bool PAGED, bool CAND, bool BAL>
 __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int b, int m, int rem) {
   Item it;
   it.b = b;
@@ -272,7 +272,7 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
     it.n_main = last >= 0 ? (int)(last / BN) + 1 : 0;
     total = it.n_main;
   }
-  if (P.balanced) {
+  if (BAL) {
     it.s = blockIdx.x;  // the item id: where its partial sums go
     it.t0 = sm.bal_t0;
     it.t1 = min(total, sm.bal_t1);
@@ -384,11 +384,12 @@ __device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
   (void)found;
 }
 
-// The rnd-th item of this CTA: one fixed item with balanced splits, otherwise
-// the snake order over the longest-first item list.
+// The rnd-th item of this CTA: one fixed item with balanced splits (BAL),
+// otherwise the snake order over the longest-first item list.
+template <bool BAL>
 __device__ __forceinline__ bool next_item(const KParams& P, const Smem& sm, Sched<BM>& sc,
                                           long long rnd, int lane, int& b, int& m, int& rem) {
-  if (P.balanced) {
+  if (BAL) {
     if (rnd > 0 || !sm.bal_ok) return false;
     b = sm.bal_b;
     m = sm.bal_m;
@@ -508,7 +509,9 @@ __device__ __forceinline__ void pw_chunk_any(const uint32_t (&sv)[16], uint32_t 
 }
 
 // ------------------------------------------------------------ the kernel
-template <bool PAGED, bool CAND, bool PW2>
+// BAL: balanced key splits (one item per CTA, compact partial blocks); only
+// paged launches split keys.
+template <bool PAGED, bool CAND, bool PW2, bool BAL>
 __global__ void __launch_bounds__(kThreads, 1)
     hstu_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -603,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
   }
   __syncthreads();
-  if (P.balanced && warp == 0) plan_balanced<CAND>(P, sm, lane);
+  if (BAL && warp == 0) plan_balanced<CAND>(P, sm, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -618,8 +621,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
       int b, m, rem;
-      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
         const uint32_t qs = qi % QST;
@@ -723,8 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       const int nt = it.t1 - it.t0;
       if (lane == 0) {
@@ -800,12 +803,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
         int b, m, rem;
-        if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
-        const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+        if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+        const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
         if (it.t0 >= it.t1) continue;
         const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
+        // Key timestamps run two tiles ahead of their slots: the loads of tiles
+        // i + 1 and i + 2 are in flight while tile i waits for its slot and is
+        // converted, so one global-load latency is not paid per tile.  Lanes
+        // past the user's keys load nothing and take the base value later.
+        long long ka[BN / 32], kb[BN / 32];
+        auto load_tile = [&](int tile, long long (&dst)[BN / 32]) {
+#pragma unroll
+          for (int i = 0; i < BN / 32; ++i) {
+            const int64_t kp = (int64_t)tile * BN + lane + 32 * i;
+            if (kp < it.n_k) dst[i] = P.ts[it.kv_row0 + kp];
+          }
+        };
+        load_tile(it.t0, ka);
+        if (it.t0 + 1 < it.t1) load_tile(it.t0 + 1, kb);
         {  // query timestamps of this item's rows
           const uint32_t qsl = qitem & 1;
+          long long qv[BM / 32];
+#pragma unroll
+          for (int i = 0; i < BM / 32; ++i) {
+            const int r = lane + 32 * i;
+            if (r < it.nvalid && it.n_k > 0) {
+              const int64_t qpc = min64(max64(it.p0 + r, 0), it.n_k - 1);
+              qv[i] = P.ts[it.kv_row0 + qpc];
+            }
+          }
           ok = mbar_wait_warp(smem_u32(&sm.qts_empty[qsl]), ((qitem >> 1) & 1) ^ 1);
           if (!ok) break;
           TsSlot& qs = sm.qts[qsl];
@@ -813,11 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < BM / 32; ++i) {
             const int r = lane + 32 * i;
-            long long v = base;
-            if (r < it.nvalid && it.n_k > 0) {
-              const int64_t qpc = min64(max64(it.p0 + r, 0), it.n_k - 1);
-              v = P.ts[it.kv_row0 + qpc];
-            }
+            const long long v = (r < it.nvalid && it.n_k > 0) ? qv[i] : base;
             const long long rel = v - base;
             exact = exact && rel > -(1LL << 23) && rel < (1LL << 23);
             qs.i[r] = v;
@@ -833,6 +855,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qitem;
         }
         for (int tile = it.t0; tile < it.t1; ++tile, ++g) {
+          long long cur[BN / 32];
+#pragma unroll
+          for (int i = 0; i < BN / 32; ++i) {
+            cur[i] = ka[i];
+            ka[i] = kb[i];
+          }
+          if (tile + 2 < it.t1) load_tile(tile + 2, kb);
           const uint32_t slot = g % NTS;
           ok = mbar_wait_warp(smem_u32(&sm.ts_empty[slot]), ((g / NTS) & 1) ^ 1);
           if (!ok) break;
@@ -842,8 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < BN / 32; ++i) {
             const int c = lane + 32 * i;
             const int64_t kp = (int64_t)tile * BN + c;
-            long long v = base;
-            if (kp < it.n_k) v = P.ts[it.kv_row0 + kp];
+            const long long v = kp < it.n_k ? cur[i] : base;
             const long long rel = v - base;
             exact = exact && rel > -(1LL << 23) && rel < (1LL << 23);
             ts.i[c] = v;
@@ -894,8 +922,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
@@ -1071,8 +1099,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (P.partial) {
           // whole 32-byte sectors when the buffer allows: the scattered
           // per-row partial stores drain faster than as 16-byte pieces
-          float* dst = P.balanced
-                           ? P.partial + ((int64_t)it.s * BM + r) * HD + ocol
+          float* dst = BAL ? P.partial + ((int64_t)it.s * BM + r) * HD + ocol
                            : P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
                                  it.h * HD + ocol;
           if (P.part_v8) {
@@ -1131,8 +1158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item(P, sm, sc, rnd, lane, b, m, rem)) break;
-      const Item it = make_item<PAGED, CAND>(P, sm, b, m, rem);
+      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
@@ -1273,8 +1300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (P.partial) {
           // whole 32-byte sectors when the buffer allows: the scattered
           // per-row partial stores drain faster than as 16-byte pieces
-          float* dst = P.balanced
-                           ? P.partial + ((int64_t)it.s * BM + r) * HD + cbase
+          float* dst = BAL ? P.partial + ((int64_t)it.s * BM + r) * HD + cbase
                            : P.partial + ((int64_t)it.s * P.total_q + row) * (int64_t)P.H * HD +
                                  it.h * HD + cbase;
           if (P.part_v8) {
@@ -1315,91 +1341,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Deterministic reduction of the key-split partials: for each query row,
-// sum the valid splits in split order, scale, round to bf16.
-template <bool PAGED>
-__global__ void split_reduce_kernel(KParams P, int B) {
+// Deterministic reduction of the balanced key splits: CTA (x, g) sums, for
+// the group g = (user b, query tile m, head h), the runs' partial blocks in run
+// order over 8 of the tile's rows (one float4 per thread), then scales and
+// rounds to bf16.  The group's items are first + (m H + h) ns .. + ns - 1
+// (plan_balanced), each a contiguous fp32 [BM, HD] block; the four metadata
+// loads are independent, so the partial loads start one memory latency after
+// the kernel does.
+constexpr int kReduceRows = 8;
+constexpr int kReduceThreads = 256;  // one float4 of one of the 8 rows per thread
+
+__global__ void __launch_bounds__(kReduceThreads) split_reduce_kernel(KParams P, int max_qt) {
   pdl_launch_dependents();
   pdl_wait();
-  const int64_t row = blockIdx.x;
-  // a launch for one chunk of users owns rows [q_off[0], q_off[B]) only: rows of
-  // other chunks are finished outputs and must not be touched
-  if (row >= P.total_q || row < P.q_off[0] || row >= P.q_off[B]) return;
-  // find the user of this row
-  int lo = 0, hi = B;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (P.q_off[mid] <= row) lo = mid;
-    else hi = mid;
-  }
-  const int b = lo;
-  const int F = P.H * HD;
-  if (P.balanced) {
-    // item (user b, query tile m, head h, run s) = plan[b] + (m H + h) ns + s
-    const int64_t rel = row - P.q_off[b];
-    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
-    const int qt = (int)((nq + BM - 1) / BM);
-    const int m = (int)(rel / BM), rr = (int)(rel % BM);
-    const int first = P.plan[b];
-    const int ns = (P.plan[b + 1] - first) / (qt * P.H);
-    for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
-      const int h = f / HD, c = f % HD;
-      const int item0 = first + (m * P.H + h) * ns;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sidx = 0; sidx < ns; ++sidx) {
-        const float4 x = *reinterpret_cast<const float4*>(
-            P.partial + ((int64_t)(item0 + sidx) * BM + rr) * HD + c);
-        acc.x += x.x;
-        acc.y += x.y;
-        acc.z += x.z;
-        acc.w += x.w;
-      }
-      __nv_bfloat16* dst = P.out + row * P.out_stride + f;
-      uint2 u;
-      u.x = pack_bf16x2(acc.x * P.scale, acc.y * P.scale);
-      u.y = pack_bf16x2(acc.z * P.scale, acc.w * P.scale);
-      *reinterpret_cast<uint2*>(dst) = u;
+  const int g = blockIdx.y;
+  const int b = g / (max_qt * P.H);
+  const int m = (g / P.H) % max_qt;
+  const int h = g % P.H;
+  if (b >= P.B) return;
+  const int64_t q0 = P.q_off[b], q1 = P.q_off[b + 1];
+  const int first = P.plan[b], next = P.plan[b + 1];
+  const int64_t nq = q1 - q0;
+  const int qt = (int)((nq + BM - 1) / BM);
+  if (m >= qt) return;
+  const int ns = (next - first) / (qt * P.H);
+  const int item0 = first + (m * P.H + h) * ns;
+  const int rr = blockIdx.x * kReduceRows + threadIdx.x / (HD / 4);
+  const int c4 = threadIdx.x % (HD / 4);
+  if (m * BM + rr >= nq) return;
+  const float* src = P.partial + ((int64_t)item0 * BM + rr) * HD + c4 * 4;
+  constexpr int64_t kBlk = (int64_t)BM * HD;  // floats between consecutive runs' blocks
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int sidx = 0;
+  // four runs' loads in flight at a time; the sums still go in run order
+  for (; sidx + 4 <= ns; sidx += 4) {
+    float4 x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[j] = *reinterpret_cast<const float4*>(src + (sidx + j) * kBlk);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc.x += x[j].x;
+      acc.y += x[j].y;
+      acc.z += x[j].z;
+      acc.w += x[j].w;
     }
-    return;
   }
-  int64_t n_k;
-  if (PAGED) {
-    const int64_t u = P.users[b];
-    n_k = (u >= 0 && u < P.max_users) ? P.lengths[u] : 0;
-  } else {
-    n_k = P.kv_off[b + 1] - P.kv_off[b];
+  for (; sidx < ns; ++sidx) {
+    const float4 x = *reinterpret_cast<const float4*>(src + sidx * kBlk);
+    acc.x += x.x;
+    acc.y += x.y;
+    acc.z += x.z;
+    acc.w += x.w;
   }
-  int total;  // key tiles of this row's item, as make_item counts them
-  if (P.mode == 1) {
-    total = (int)((n_k + BN - 1) / BN) + 1;  // candidate layout: history tiles + 1
-  } else {
-    // causal suffix: the item's tiles run up to its query tile's last row
-    const int64_t nq = P.q_off[b + 1] - P.q_off[b];
-    const int64_t m = (row - P.q_off[b]) / BM;
-    const int64_t last = n_k - nq + min64(BM * (m + 1), nq) - 1;
-    total = last >= 0 ? (int)(last / BN) + 1 : 0;
-  }
-  const int n_valid = min(P.n_split, (total + P.kps - 1) / P.kps);
-  for (int f = threadIdx.x * 4; f < F; f += blockDim.x * 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_valid; ++s) {
-      const float4 x = *reinterpret_cast<const float4*>(P.partial + ((int64_t)s * P.total_q + row) * F + f);
-      acc.x += x.x;
-      acc.y += x.y;
-      acc.z += x.z;
-      acc.w += x.w;
-    }
-    __nv_bfloat16* dst = P.out + row * P.out_stride + f;
-    uint2 u;
-    u.x = pack_bf16x2(acc.x * P.scale, acc.y * P.scale);
-    u.y = pack_bf16x2(acc.z * P.scale, acc.w * P.scale);
-    *reinterpret_cast<uint2*>(dst) = u;
-  }
+  const int64_t row = q0 + m * BM + rr;
+  if (row >= P.total_q) return;
+  __nv_bfloat16* dst = P.out + row * P.out_stride + h * HD + c4 * 4;
+  uint2 u;
+  u.x = pack_bf16x2(acc.x * P.scale, acc.y * P.scale);
+  u.y = pack_bf16x2(acc.z * P.scale, acc.w * P.scale);
+  *reinterpret_cast<uint2*>(dst) = u;
 }
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-template <bool PAGED, bool CAND, bool PW2 = false>
+template <bool PAGED, bool CAND, bool PW2 = false, bool BAL = false>
 cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items, int num_sms,
                         cudaStream_t stream) {
   CUtensorMap tq, tk, tv, tkc, tvc;
@@ -1426,7 +1431,8 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     tkc = tq;
     tvc = tq;
   }
-  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PW2>;
+  static_assert(PAGED || !BAL, "only paged launches split keys");
+  auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PW2, BAL>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1441,8 +1447,9 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
   cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq, tk,
                                    tv, tkc, tvc, kp);
   if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
-  return launch_dependent(split_reduce_kernel<PAGED>, dim3((unsigned)p.total_q), dim3(128), 0, stream,
-                          kp, p.B);
+  const int max_qt = std::max(1, (p.max_q + BM - 1) / BM);
+  return launch_dependent(split_reduce_kernel, dim3(BM / kReduceRows, (unsigned)(p.B * p.H * max_qt)),
+                          dim3(kReduceThreads), 0, stream, kp, max_qt);
 }
 
 // Key-split plan: one wave of (user, head, split) items, each streaming a long
@@ -1548,12 +1555,13 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
   kp.total_q = p.total_q;
   kp.err = err_word;
   long long items_override = -1;
+  bool balanced = false;
   if (kp.n_split > 1 || p.partial_only) {
     const size_t need = attn_sm100_workspace_bytes(p, num_sms);
     if (workspace == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
     if (!p.partial_only) {
       // balanced splits, one item per CTA (the kernel chooses the runs)
-      kp.balanced = 1;
+      balanced = true;
       kp.n_split = 1;
       kp.kps = 1 << 30;
       kp.plan = reinterpret_cast<int*>(workspace);
@@ -1569,10 +1577,13 @@ cudaError_t attn_sm100_launch(const AttnProblem& p, void* workspace, size_t ws_b
   const long long items =
       items_override > 0 ? items_override : (long long)p.B * p.H * std::max(qt, 1) * kp.n_split;
   if (p.paged) {
-    if (p.mode == 1) return launch_impl<true, true>(p, kp, items, num_sms, stream);
+    if (p.mode == 1)
+      return balanced ? launch_impl<true, true, false, true>(p, kp, items, num_sms, stream)
+                         : launch_impl<true, true, false, false>(p, kp, items, num_sms, stream);
     // paged causal attention (the long-history path) runs the two-pair
     // pointwise layout: measured faster there than 16 warps per tile
-    return launch_impl<true, false, true>(p, kp, items, num_sms, stream);
+    return balanced ? launch_impl<true, false, true, true>(p, kp, items, num_sms, stream)
+                       : launch_impl<true, false, true, false>(p, kp, items, num_sms, stream);
   }
   return p.mode == 1 ? launch_impl<false, true>(p, kp, items, num_sms, stream)
                      : launch_impl<false, false>(p, kp, items, num_sms, stream);

@@ -10,12 +10,12 @@
 // bf16 storage, fp32 accumulation; UVQK, A, G and X are the bf16 tensors the
 // stack materialises.
 //
-// GEMM kernel: persistent, one CTA per SM, 192 threads.  Warp 0 issues TMA
+// GEMM kernel: persistent, one CTA per SM, 320 threads.  Warp 0 issues TMA
 // (A tile 128 x 64 K-major, B tile 64 x 256 MN-major, 128-byte swizzle, 4
 // stages), warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two
-// TMEM accumulators (2 x 256 columns), warps 2-5 drain the other accumulator
-// (tcgen05.ld -> epilogue -> global) so the epilogue of tile i overlaps the
-// main loop of tile i+1.
+// TMEM accumulators (2 x 256 columns), warps 2-9 drain the other accumulator
+// (tcgen05.ld -> epilogue -> global; two warps per TMEM lane quarter, 128
+// columns each) so the epilogue of tile i overlaps the main loop of tile i+1.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -32,7 +32,9 @@ namespace {
 
 constexpr int GBM = 128, GBN = 256, GBK = 64;
 constexpr int GST = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
+constexpr int kEpiWarps = 8;                 // warps 2..9
+constexpr int kEpiCols = GBN / 2;            // columns per epilogue warp
 constexpr int kABytes = GBM * GBK * 2;       // 16 KiB
 constexpr int kBBytes = GBK * GBN * 2;       // 32 KiB
 constexpr int kBBoxBytes = GBK * 64 * 2;     // one 64-column B box: 8 KiB
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.acc_full[i]), 1);
-      mbar_init(smem_u32(&sm.acc_empty[i]), 4);
+      mbar_init(smem_u32(&sm.acc_empty[i]), kEpiWarps);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
     fence_mbar_init();
@@ -153,8 +155,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else {
-    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // epilogue warps 2..9: TMEM lane quarter = warp % 4, column half by warp
     const int sub = warp & 3;
+    const int chalf = (warp - 2) >> 2;
     const int r = sub * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     uint32_t tcount = 0;
@@ -163,15 +166,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t ab = tcount & 1;
       const int64_t row = (int64_t)mt * GBM + r;
       const bool valid = row < P.M;
-      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN;
+      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN + chalf * kEpiCols;
       // residual epilogue: this thread's whole row segment of X is loaded
       // before the accumulator is ready (one memory latency per tile, hidden
       // behind the main loop, instead of one per 32-column chunk)
-      uint4 res[EPI == EPI_RESIDUAL ? GBN / 8 : 1];
+      uint4 res[EPI == EPI_RESIDUAL ? kEpiCols / 8 : 1];
       if (EPI == EPI_RESIDUAL && valid) {
         const uint4* src = reinterpret_cast<const uint4*>(orow);
 #pragma unroll
-        for (int q = 0; q < GBN / 8; ++q) res[q] = src[q];
+        for (int q = 0; q < kEpiCols / 8; ++q) res[q] = src[q];
       }
       if (!mbar_wait_warp(smem_u32(&sm.acc_full[ab]), (tcount >> 1) & 1)) {
         if (lane == 0) atomicExch(P.err, DEV_ERR_TIMEOUT);
@@ -179,12 +182,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < GBN / 32; ++ch) {
+      for (int ch = 0; ch < kEpiCols / 32; ++ch) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_addr + ab * GBN + ch * 32, v);
+        tmem_ld32(tmem + lane_addr + ab * GBN + chalf * kEpiCols + ch * 32, v);
         tmem_wait_ld();
         reg_fence(v);
-        if (ch == GBN / 32 - 1) {
+        if (ch == kEpiCols / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.acc_empty[ab]));

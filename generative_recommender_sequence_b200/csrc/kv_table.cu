@@ -209,10 +209,64 @@ __global__ void __launch_bounds__(kAllocThreads)
 // 16-byte vectors, so 256 threads copy two tokens with one vector each
 constexpr int kAppendTok = 2;
 constexpr int kCopyThreads = 256;
+// tokens per CTA of a bulk append (a prefill or an onboarding): whole 32-token
+// pages' worth of K and V per CTA instead of two tokens
+constexpr int kBulkTok = 64;
+constexpr int kBulkFromTokens = 256;  // bulk CTAs once some user appends this many
+// tokens per CTA of the one-launch serving step (each thread's vectors are
+// loaded before the plan resolves); measured: 2 tokens per CTA beat 8 on the
+// serving steps (more CTAs in flight outweigh the completion-counter traffic)
+constexpr int kStepTok = 2;
+constexpr int kStepVec = kStepTok * 2 * 64 / kCopyThreads;  // bf16 H=4 d=128: 16-byte vectors per thread
 
-// grid (chunks, B): CTA (c, b) copies tokens [c*kAppendTok, ...) of user b.
+// Copies ntok consecutive tokens (source rows src_row0.., positions p0..) of
+// K and V into their pages (s_page[i] = page of position (first_page + i) *
+// page_size ..).  Thread-strided over 16-byte vectors, eight loads in flight
+// per thread before their stores.  H_, D_, PS_ != 0 fix the layout at compile
+// time (shifts instead of divisions); 0 reads it from the table.
+template <int ESZ, int H_, int D_, int PS_>
+__device__ __forceinline__ void bulk_copy(const KvTableDev& t, const uint8_t* __restrict__ k_new,
+                                          const uint8_t* __restrict__ v_new, int64_t src_row0,
+                                          int64_t src_row_bytes, int ntok, int64_t p0,
+                                          int64_t first_page, const int32_t* s_page) {
+  const int H = H_ ? H_ : t.H, D = D_ ? D_ : t.d, PS = PS_ ? PS_ : t.page_size;
+  const int vph = D * ESZ / 16;  // 16-byte vectors per head row
+  const int row_vec = H * vph;
+  const int total = ntok * row_vec * 2;
+  constexpr int U = 8;
+  for (int base = threadIdx.x; base < total; base += kCopyThreads * U) {
+    uint4 x[U];
+    int64_t dst_off[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int i = base + j * kCopyThreads;
+      dst_off[j] = -1;
+      if (i < total) {
+        const int kv = i / (ntok * row_vec);
+        const int rem = i - kv * (ntok * row_vec);
+        const int tk = rem / row_vec, v = rem - tk * row_vec;
+        const int h = v / vph, e16 = v - h * vph;
+        const int64_t pos = p0 + tk;
+        const int32_t page = s_page[(int)(pos / PS - first_page)];
+        const int slot = (int)(pos % PS);
+        const uint8_t* src = (kv ? v_new : k_new) + (src_row0 + tk) * src_row_bytes;
+        x[j] = reinterpret_cast<const uint4*>(src)[v];
+        dst_off[j] = ((((int64_t)page * 2 + kv) * H + h) * PS + slot) * D * ESZ + (int64_t)e16 * 16;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j)
+      if (dst_off[j] >= 0)
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(t.pool) + dst_off[j]) = x[j];
+  }
+}
+
+// grid (chunks, B): CTA (c, b) copies tokens [c*TOK, ...) of user b (TOK =
+// kAppendTok for serving-sized appends, kBulkTok for prefills and onboarding).
 // The length is read before any copy and advanced by the last CTA of the user.
-template <int ESZ>
+// A bulk CTA first reads the (at most two) pages its tokens land in, then
+// copies with every thread's loads in flight before its stores.
+template <int ESZ, int TOK>
 __global__ void __launch_bounds__(kCopyThreads)
     kv_append_kernel(KvTableDev t, const int64_t* __restrict__ users,
                      const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
@@ -222,7 +276,7 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int b = blockIdx.y;
   const int64_t u = users[b];
   const int64_t s = new_offsets[b], n = new_offsets[b + 1] - s;
-  const int n_chunks = (int)((n + kAppendTok - 1) / kAppendTok);
+  const int n_chunks = (int)((n + TOK - 1) / TOK);
   if (blockIdx.x >= n_chunks) return;
   if (u < 0 || u >= t.max_users) {
     if (threadIdx.x == 0) set_status(t.status, 1);
@@ -233,22 +287,40 @@ __global__ void __launch_bounds__(kCopyThreads)
   if (fits) {
     const int row_vec = t.H * t.d * ESZ / 16;     // 16-byte vectors per token row
     const int vec_per_head = t.d * ESZ / 16;
-    const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
-    const int ntok = (int)((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok);
-    for (int i = threadIdx.x; i < ntok * row_vec * 2; i += kCopyThreads) {
-      const int kv = i / (ntok * row_vec);
-      const int rem = i % (ntok * row_vec);
-      const int tk = rem / row_vec, v = rem % row_vec;
-      const int h = v / vec_per_head, e16 = v % vec_per_head;
-      const int64_t src_row = s + tok0 + tk;
-      const int64_t pos = len + tok0 + tk;
-      const int32_t page = t.page_lists[u * (int64_t)t.max_ppu + pos / t.page_size];
-      const int slot = (int)(pos % t.page_size);
-      const uint8_t* src = (kv ? v_new : k_new) + src_row * src_row_bytes;
-      const uint4 x = reinterpret_cast<const uint4*>(src)[v];
-      uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
-                     ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
-      reinterpret_cast<uint4*>(dst)[e16] = x;
+    const int64_t tok0 = (int64_t)blockIdx.x * TOK;
+    const int ntok = (int)((n - tok0) < TOK ? (n - tok0) : TOK);
+    const int32_t* plist = t.page_lists + u * (int64_t)t.max_ppu;
+    if (TOK <= kAppendTok) {
+      for (int i = threadIdx.x; i < ntok * row_vec * 2; i += kCopyThreads) {
+        const int kv = i / (ntok * row_vec);
+        const int rem = i % (ntok * row_vec);
+        const int tk = rem / row_vec, v = rem % row_vec;
+        const int h = v / vec_per_head, e16 = v % vec_per_head;
+        const int64_t src_row = s + tok0 + tk;
+        const int64_t pos = len + tok0 + tk;
+        const int32_t page = plist[pos / t.page_size];
+        const int slot = (int)(pos % t.page_size);
+        const uint8_t* src = (kv ? v_new : k_new) + src_row * src_row_bytes;
+        const uint4 x = reinterpret_cast<const uint4*>(src)[v];
+        uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
+                       ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
+        reinterpret_cast<uint4*>(dst)[e16] = x;
+      }
+    } else {
+      // the chunk's positions span pages first_page .. first_page + n_pg - 1
+      __shared__ int32_t s_page[kBulkTok / 32 + 2];
+      const int64_t p0 = len + tok0;
+      const int64_t first_page = p0 / t.page_size;
+      const int n_pg = (int)((p0 + ntok - 1) / t.page_size - first_page) + 1;
+      for (int i = threadIdx.x; i < n_pg; i += kCopyThreads) s_page[i] = plist[first_page + i];
+      __syncthreads();
+      // the common layout (bf16, 4 heads of 128) gets compile-time strides
+      if (ESZ == 2 && t.H == 4 && t.d == 128 && t.page_size == 32)
+        bulk_copy<ESZ, 4, 128, 32>(t, k_new, v_new, s + tok0, src_row_bytes, ntok, p0, first_page,
+                                   s_page);
+      else
+        bulk_copy<ESZ, 0, 0, 0>(t, k_new, v_new, s + tok0, src_row_bytes, ntok, p0, first_page,
+                                s_page);
     }
   } else if (threadIdx.x == 0 && blockIdx.x == 0) {
     set_status(t.status, 1);
@@ -353,21 +425,26 @@ __global__ void __launch_bounds__(kCopyThreads)
   int held, need = 0, pre = 0;
   const int64_t s0 = new_offsets[b];
   const int64_t n = new_offsets[b + 1] - s0;
-  // this thread's first source vector depends on nothing the plan computes:
-  // load it now so its latency overlaps the plan's dependent loads
+  // this thread's first source vectors depend on nothing the plan computes:
+  // load them now so their latency overlaps the plan's dependent loads
   const int row_vec = t.H * t.d * ESZ / 16;  // 16-byte vectors per token row
-  const int64_t tok0 = (int64_t)blockIdx.x * kAppendTok;
+  const int64_t tok0 = (int64_t)blockIdx.x * kStepTok;
   // (a count above max_new makes the batch invalid: nothing is read for it,
   // and the buffers may then be null)
   const int ntok = (int)(tok0 < n && n <= max_new
-                             ? ((n - tok0) < kAppendTok ? (n - tok0) : kAppendTok)
+                             ? ((n - tok0) < kStepTok ? (n - tok0) : kStepTok)
                              : 0);
-  uint4 x0 = make_uint4(0u, 0u, 0u, 0u);
-  if (tid < ntok * row_vec * 2) {
-    const int kv = tid / (ntok * row_vec);
-    const int rem = tid % (ntok * row_vec);
-    const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + rem / row_vec) * src_row_bytes;
-    x0 = reinterpret_cast<const uint4*>(src)[rem % row_vec];
+  uint4 xpre[kStepVec];
+#pragma unroll
+  for (int j = 0; j < kStepVec; ++j) {
+    const int i = tid + j * kCopyThreads;
+    xpre[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < ntok * row_vec * 2) {
+      const int kv = i / (ntok * row_vec);
+      const int rem = i % (ntok * row_vec);
+      const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + rem / row_vec) * src_row_bytes;
+      xpre[j] = reinterpret_cast<const uint4*>(src)[rem % row_vec];
+    }
   }
   if (PLAN) {
     if (tid == 0) {
@@ -453,26 +530,33 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int32_t* list = t.page_lists + (known ? u : 0) * (int64_t)t.max_ppu;
   if (ok && tok0 < n) {
     const int vec_per_head = t.d * ESZ / 16;
-    for (int i = tid; i < ntok * row_vec * 2; i += kCopyThreads) {
+    const int total = ntok * row_vec * 2;
+    // where vector i goes: pages this step pops come straight from the stack
+    // (PLAN); the rest are on the user's list
+    auto dst_of = [&](int i) -> uint4* {
       const int kv = i / (ntok * row_vec);
       const int rem = i % (ntok * row_vec);
       const int tk = rem / row_vec, v = rem % row_vec;
       const int h = v / vec_per_head, e16 = v % vec_per_head;
       const int64_t pos = len + tok0 + tk;
       const int64_t pi = pos / t.page_size;
-      // pages this step pops come straight from the stack (PLAN); the rest
-      // are on the user's list
       const int32_t page = (PLAN && pi >= held) ? t.free_stack[top - 1 - (pre + (pi - held))]
                                                 : list[pi];
       const int slot = (int)(pos % t.page_size);
-      uint4 x = x0;
-      if (i != tid) {
-        const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + tk) * src_row_bytes;
-        x = reinterpret_cast<const uint4*>(src)[v];
-      }
       uint8_t* dst = reinterpret_cast<uint8_t*>(t.pool) +
                      ((((int64_t)page * 2 + kv) * t.H + h) * t.page_size + slot) * t.d * ESZ;
-      reinterpret_cast<uint4*>(dst)[e16] = x;
+      return reinterpret_cast<uint4*>(dst) + e16;
+    };
+#pragma unroll
+    for (int j = 0; j < kStepVec; ++j) {
+      const int i = tid + j * kCopyThreads;
+      if (i < total) *dst_of(i) = xpre[j];
+    }
+    for (int i = tid + kStepVec * kCopyThreads; i < total; i += kCopyThreads) {
+      const int kv = i / (ntok * row_vec);
+      const int rem = i % (ntok * row_vec);
+      const uint8_t* src = (kv ? v_new : k_new) + (s0 + tok0 + rem / row_vec) * src_row_bytes;
+      *dst_of(i) = reinterpret_cast<const uint4*>(src)[rem % row_vec];
     }
   }
   if (blockIdx.x == 0) {
@@ -514,7 +598,7 @@ __global__ void __launch_bounds__(kCopyThreads)
     __threadfence();
   } else {
     // the last CTA of this user commits the new length
-    const int n_chunks = (int)((n + kAppendTok - 1) / kAppendTok);
+    const int n_chunks = (int)((n + kStepTok - 1) / kStepTok);
     if (tid == 0 && tok0 < n) {
       __threadfence();
       const int prev = atomicAdd(&t.done[u], 1);
@@ -627,12 +711,22 @@ cudaError_t kv_append_launch(const KvTableDev& t, const int64_t* users, const vo
   // 16-byte vector copies: every source row must start on a 16-byte boundary
   if (row_elems < (int64_t)t.H * t.d || (row_elems * t.esize) % 16 != 0)
     return cudaErrorInvalidValue;
-  dim3 grid((max_new + kAppendTok - 1) / kAppendTok, B);
+  const uint8_t* k = (const uint8_t*)k_new;
+  const uint8_t* v = (const uint8_t*)v_new;
+  if (max_new >= kBulkFromTokens) {
+    const dim3 grid((max_new + kBulkTok - 1) / kBulkTok, B);
+    if (t.esize == 2)
+      return launch_dependent(kv_append_kernel<2, kBulkTok>, grid, dim3(kCopyThreads), 0, stream, t,
+                              users, k, v, new_offsets, row_elems * 2);
+    return launch_dependent(kv_append_kernel<4, kBulkTok>, grid, dim3(kCopyThreads), 0, stream, t,
+                            users, k, v, new_offsets, row_elems * 4);
+  }
+  const dim3 grid((max_new + kAppendTok - 1) / kAppendTok, B);
   if (t.esize == 2)
-    return launch_dependent(kv_append_kernel<2>, grid, dim3(kCopyThreads), 0, stream, t, users,
-                            (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 2);
-  return launch_dependent(kv_append_kernel<4>, grid, dim3(kCopyThreads), 0, stream, t, users,
-                          (const uint8_t*)k_new, (const uint8_t*)v_new, new_offsets, row_elems * 4);
+    return launch_dependent(kv_append_kernel<2, kAppendTok>, grid, dim3(kCopyThreads), 0, stream, t,
+                            users, k, v, new_offsets, row_elems * 2);
+  return launch_dependent(kv_append_kernel<4, kAppendTok>, grid, dim3(kCopyThreads), 0, stream, t,
+                          users, k, v, new_offsets, row_elems * 4);
 }
 
 cudaError_t kv_lookup_launch(const KvTableDev& t, const int64_t* users, int B,
@@ -661,7 +755,7 @@ cudaError_t kv_step_launch(const KvTableDev& t, const int64_t* users, const void
   if (row_elems < (int64_t)t.H * t.d || (row_elems * t.esize) % 16 != 0)
     return cudaErrorInvalidValue;
   if (page_table_out == nullptr) max_pages = 0;
-  const dim3 grid(std::max(1, (max_new + kAppendTok - 1) / kAppendTok), B);
+  const dim3 grid(std::max(1, (max_new + kStepTok - 1) / kStepTok), B);
   const int64_t rb = row_elems * t.esize;
   const uint8_t* k = (const uint8_t*)k_new;
   const uint8_t* v = (const uint8_t*)v_new;

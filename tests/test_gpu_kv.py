@@ -214,3 +214,48 @@ def test_kv_release_bit_exact_through_later_allocations():
     t.lookup(dev(users.astype(np.int64)), lens2)
     assert np.array_equal(lens2.cpu().numpy(), rl) and t.storage() == before
     t.close()
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_kv_bulk_append_bit_exact(dtype, d):
+    """Prefill-sized appends (64 tokens per CTA, from 256 new tokens on) onto
+    lengths that end mid-page, interleaved with serving-sized ones: page ids,
+    lookups and pool bytes match the sequential oracle bit for bit."""
+    import generative_recommender_sequence_b200 as hstu
+    rng = np.random.default_rng(9)
+    n_pages, H, U = 400, 2, 6
+    order = rng.permutation(n_pages)
+    t = hstu.KVTable(n_pages, H, d, dtype=dtype, max_users=U, max_pages_per_user=128,
+                     free_order=order)
+    ref = KVTableOracle(n_pages, 32, H, d, U, 128, order,
+                        dtype="bf16" if dtype == torch.bfloat16 else "f32")
+    sizes = [[37, 1500, 5], [300, 0, 700], [3, 2, 1], [256, 255, 1029]]
+    for n_list in sizes:
+        users = rng.permutation(U)[:len(n_list)]
+        n = np.array(n_list, np.int64)
+        t.alloc(dev(users.astype(np.int64)), dev(n))
+        rs, _ = ref.alloc(users.tolist(), n.tolist())
+        assert t.status() == rs == OK
+        kv = rng.standard_normal((2, int(n.sum()), H, d)).astype(np.float32)
+        if dtype == torch.bfloat16:
+            kv = workloads._as_storage(kv, "bf16")
+        off = workloads.offsets_from_lengths(n)
+        st = "bf16" if dtype == torch.bfloat16 else "f32"
+        t.append(dev(users.astype(np.int64)), storage(kv[0], st), storage(kv[1], st), dev(off),
+                 int(max(n.max(), 1)))
+        assert t.status() == OK
+        assert ref.append(users.tolist(), kv[0], kv[1], off) == OK
+    users = np.arange(U)
+    rl, rt, rk, rv = ref.lookup(users.tolist(), 128)
+    lens = torch.empty(U, dtype=torch.int64, device="cuda")
+    table = torch.empty((U, 128), dtype=torch.int32, device="cuda")
+    out_off = workloads.offsets_from_lengths(rl)
+    ko = torch.empty((int(out_off[-1]), H, d), dtype=dtype, device="cuda")
+    vo = torch.empty_like(ko)
+    t.lookup(dev(users.astype(np.int64)), lens, table, ko, vo, dev(out_off), int(rl.max()))
+    assert t.status() == OK
+    assert np.array_equal(lens.cpu().numpy(), rl) and np.array_equal(table.cpu().numpy(), rt)
+    bits = (lambda x: x.cpu().view(torch.int16).numpy().view(np.uint16)) if dtype == torch.bfloat16 \
+        else (lambda x: x.cpu().view(torch.int32).numpy().view(np.uint32))
+    assert np.array_equal(bits(ko), rk) and np.array_equal(bits(vo), rv)
+    t.close()
