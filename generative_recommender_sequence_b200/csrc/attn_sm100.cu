@@ -286,7 +286,7 @@ __device__ __forceinline__ Item make_item(const KParams& P, const Smem& sm, int 
   return it;
 }
 
-__device__ __forceinline__ long long warp_sum_ll(long long v) {
+__device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -296,14 +296,14 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
 // candidate user; causal runs in this mode have at most one query tile) and
 // its number of query tiles.
 template <bool CAND>
-__device__ __forceinline__ int plan_tiles(const KParams& P, const Smem& sm, int b, int& qt) {
+__device__ __forceinline__ int plan_tiles(const Smem& sm, int b, int& qt) {
   const int nq = sm.m_q[b + 1] - sm.m_q[b];
-  const int64_t n_k = sm.m_nk[b];
+  const int n_k = sm.m_nk[b];
   qt = nq > 0 ? (nq + BM - 1) / BM : 0;
   if (qt == 0) return 0;
-  if (CAND) return (int)((n_k + BN - 1) / BN) + 1;
-  const int64_t last = n_k - nq + min64(BM, nq) - 1;
-  return last >= 0 ? (int)(last / BN) + 1 : 0;
+  if (CAND) return (n_k + BN - 1) / BN + 1;
+  const int last = n_k - nq + min(BM, nq) - 1;
+  return last >= 0 ? last / BN + 1 : 0;
 }
 
 // Runs a user's key tiles are cut into for a target run length (round to
@@ -317,71 +317,70 @@ __device__ __forceinline__ int plan_runs(int tiles, int target) {
 // fewer (user, head, query tile) items than CTAs).  Every CTA derives the same
 // plan from the key counts: the target run length is the smallest that is at
 // least ceil(total tiles / CTAs) and lets every user's runs fit one wave, user
-// b's tiles are cut into plan_runs(tiles_b, target) near-equal runs, and items
-// are numbered user by user, then query tile, head and run.  This CTA takes
-// item blockIdx.x; CTA 0 also publishes each user's first item for the reduce.
-// Called by warp 0 only.
+// b's tiles are cut into plan_runs(tiles_b, target) near-equal runs (the
+// first tiles_b mod runs of them one tile longer), and items are numbered user
+// by user, then query tile, head and run.  This CTA takes item blockIdx.x; CTA
+// 0 also publishes each user's first item for the reduce.  Called by warp 0
+// only; 32-bit arithmetic throughout (this runs before any copy is issued, so
+// its length is the launch's latency; the host admits this mode only with at
+// most num_sms / 2 (user, head, query tile) items).
 template <bool CAND>
 __device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
   const int G = gridDim.x;
-  long long W = 0;
-  for (int b0 = 0; b0 < P.B; b0 += 32) {
-    const int b = b0 + lane;
+  int W = 0;
+  for (int b = lane; b < P.B; b += 32) {
     int qt = 0;
-    const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
-    W += (long long)qt * P.H * t;
+    const int t = plan_tiles<CAND>(sm, b, qt);
+    W += qt * P.H * t;
   }
-  W = warp_sum_ll(W);
-  int target = (int)max(2LL, (W + G - 1) / G);
+  W = warp_sum_i(W);
+  int target = max(2, (W + G - 1) / G);
   for (int iter = 0;; ++iter) {
-    long long items = 0;
-    for (int b0 = 0; b0 < P.B; b0 += 32) {
-      const int b = b0 + lane;
+    int items = 0;
+    for (int b = lane; b < P.B; b += 32) {
       int qt = 0;
-      const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
-      items += (long long)qt * P.H * plan_runs(t, target);
+      const int t = plan_tiles<CAND>(sm, b, qt);
+      items += qt * P.H * plan_runs(t, target);
     }
-    items = warp_sum_ll(items);
+    items = warp_sum_i(items);
     if (items <= G) break;
     // one run per user always fits (the host chooses this mode only then)
     target = iter < 64 ? target + 1 : (1 << 30);
   }
   // this CTA's item: exclusive prefix of the users' item counts
-  const long long me = blockIdx.x;
-  long long base = 0;
-  bool found = false;
+  const int me = blockIdx.x;
+  int base = 0;
   if (lane == 0) sm.bal_ok = 0;
   __syncwarp();
   for (int b0 = 0; b0 < P.B; b0 += 32) {
     const int b = b0 + lane;
     int qt = 0;
-    const int t = b < P.B ? plan_tiles<CAND>(P, sm, b, qt) : 0;
+    const int t = b < P.B ? plan_tiles<CAND>(sm, b, qt) : 0;
     const int ns = plan_runs(t, target);
-    const long long cnt = (long long)qt * P.H * ns;
-    long long incl = cnt;
+    const int cnt = qt * P.H * ns;
+    int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    const long long first = base + incl - cnt;
-    if (blockIdx.x == 0 && b < P.B) P.plan[b] = (int)first;
+    const int first = base + incl - cnt;
+    if (blockIdx.x == 0 && b < P.B) P.plan[b] = first;
     if (b < P.B && cnt > 0 && me >= first && me < first + cnt) {
-      const int r = (int)(me - first);
+      const int r = me - first;
       const int per = P.H * ns;
-      const int h = (r % per) / ns, sidx = r % ns;
+      const int sidx = r % ns;
+      const int q = t / ns, rr = t % ns;   // runs of q + 1 tiles, then of q
       sm.bal_b = b;
       sm.bal_m = r / per;
-      sm.bal_h = h;
-      sm.bal_t0 = (int)((long long)sidx * t / ns);
-      sm.bal_t1 = (int)((long long)(sidx + 1) * t / ns);
+      sm.bal_h = (r % per) / ns;
+      sm.bal_t0 = sidx * q + min(sidx, rr);
+      sm.bal_t1 = sm.bal_t0 + q + (sidx < rr ? 1 : 0);
       sm.bal_ok = 1;
-      found = true;
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  if (blockIdx.x == 0 && lane == 0) P.plan[P.B] = (int)base;
-  (void)found;
+  if (blockIdx.x == 0 && lane == 0) P.plan[P.B] = base;
 }
 
 // The rnd-th item of this CTA: one fixed item with balanced splits (BAL),
@@ -616,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // =============================================== TMA producer
     Sched<BM> sc;
-    sc.init(sm.m_q, P.B, HS, lane);
+    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
@@ -720,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
     // tensor pipe fed: while one waits on its barriers the other's MMAs run.
     Sched<BM> sc;
-    sc.init(sm.m_q, P.B, HS, lane);
+    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
@@ -798,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // time-gap bias, so the pointwise warps never wait on global loads.
     if (P.time_table != nullptr && !PAGED && !CAND) {
       Sched<BM> sc;
-      sc.init(sm.m_q, P.B, HS, lane);
+      if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
       uint32_t g = 0, qitem = 0;
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
@@ -917,7 +916,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pb_idx = -1;
     float pb_val = 0.f;
     Sched<BM> sc;
-    sc.init(sm.m_q, P.B, HS, lane);
+    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0, my_epi = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
@@ -1153,7 +1152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pb_idx = -1;
     float pb_val = 0.f;
     Sched<BM> sc;
-    sc.init(sm.m_q, P.B, HS, lane);
+    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
