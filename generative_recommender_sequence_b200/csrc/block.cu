@@ -30,22 +30,30 @@
 namespace hstu {
 namespace {
 
-constexpr int GBM = 128, GBN = 256, GBK = 64;
-constexpr int GST = 4;
+constexpr int GBM = 128, GBK = 64;
 constexpr int kGemmThreads = 320;
 constexpr int kEpiWarps = 8;                 // warps 2..9
-constexpr int kEpiCols = GBN / 2;            // columns per epilogue warp
 constexpr int kABytes = GBM * GBK * 2;       // 16 KiB
-constexpr int kBBytes = GBK * GBN * 2;       // 32 KiB
 constexpr int kBBoxBytes = GBK * 64 * 2;     // one 64-column B box: 8 KiB
-constexpr uint32_t kIdescGemm = idesc_bf16_f32(GBM, GBN, true);
+
+// Tile width BN (256 for the wide projection, 128 for the 512-column output
+// projection, whose 128 x 256 tiles would give 148 SMs only 1.4 waves) and the
+// TMA ring depth that keeps about 192 KiB of operands in flight.
+template <int BN>
+struct GemmCfg {
+  static constexpr int kBBytes = GBK * BN * 2;
+  static constexpr int kStages = BN >= 256 ? 4 : 6;
+  static constexpr int kEpiCols = BN / 2;    // columns per epilogue warp
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(GBM, BN, true);
+};
 
 enum { EPI_SILU = 0, EPI_RESIDUAL = 1 };
 
+template <int BN>
 struct __align__(1024) GemmSmem {
-  uint8_t a[GST][kABytes];
-  uint8_t b[GST][kBBytes];
-  uint64_t full[GST], empty[GST];
+  uint8_t a[GemmCfg<BN>::kStages][kABytes];
+  uint8_t b[GemmCfg<BN>::kStages][GemmCfg<BN>::kBBytes];
+  uint64_t full[GemmCfg<BN>::kStages], empty[GemmCfg<BN>::kStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -58,13 +66,18 @@ struct GemmParams {
   int* err;
 };
 
-template <int EPI>
+template <int EPI, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b, const GemmParams P) {
+  constexpr int GBN = BN;
+  constexpr int GST = GemmCfg<BN>::kStages;
+  constexpr int kBBytes = GemmCfg<BN>::kBBytes;
+  constexpr int kEpiCols = GemmCfg<BN>::kEpiCols;
+  constexpr uint32_t kIdescGemm = GemmCfg<BN>::kIdesc;
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+  GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // dependent launch: barrier set-up and the TMEM allocation overlap the
   // previous kernel's tail; global memory is touched only after the wait
@@ -287,11 +300,12 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
+template <int BN>
+size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN>) + 1024; }
 
 // out[M, N] (ld ldo) = epi(A[M, K] (ld lda) @ B[K, N] (ld ldb)); residual
 // epilogue reads out before writing it.
-template <int EPI>
+template <int EPI, int GBN>
 cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb, void* out,
                         int64_t ldo, int M, int N, int K, int* err, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
@@ -301,20 +315,21 @@ cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb,
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, Bw, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 2, 64, GBK))
     return cudaErrorInvalidValue;
-  auto kern = gemm_bf16_kernel<EPI>;
+  auto kern = gemm_bf16_kernel<EPI, GBN>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm_smem_bytes());
+                                         (int)gemm_smem_bytes<GBN>());
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int tiles = ((M + GBM - 1) / GBM) * (N / GBN);
   const int grid = std::max(1, std::min(tiles, device_sm_count()));
   GemmParams p{M, N, K, reinterpret_cast<__nv_bfloat16*>(out), ldo, err};
-  return launch_dependent(kern, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(), stream, ta, tb, p);
+  return launch_dependent(kern, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<GBN>(), stream, ta,
+                          tb, p);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -338,7 +353,7 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
       reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)p.T * 4 * F * 2) + align256((size_t)p.T * F * 2));
   const int M = (int)p.T;
   for (int l = 0; l < p.n_layers; ++l) {
-    cudaError_t e = gemm_launch<EPI_SILU>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+    cudaError_t e = gemm_launch<EPI_SILU, 256>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
                                           p.d_model, err_word, stream);
     if (e != cudaSuccess) return e;
     AttnProblem a;
@@ -368,7 +383,7 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
     e = launch_dependent(ln_gate_kernel, dim3((unsigned)((p.T + 7) / 8)), dim3(256), 0, stream,
                          attn, uvqk, 4 * F, gate, p.T, p.ln_eps);
     if (e != cudaSuccess) return e;
-    e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+    e = gemm_launch<EPI_RESIDUAL, 128>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
                                   err_word, stream);
     if (e != cudaSuccess) return e;
   }
@@ -456,7 +471,7 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
   for (int l = 0; l < p.n_layers; ++l) {
     const KvTableDev& t = p.tables[l];
     // [U | V | Q | K] = SiLU(X W1) for the new and the candidate rows at once
-    cudaError_t e = gemm_launch<EPI_SILU>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+    cudaError_t e = gemm_launch<EPI_SILU, 256>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
                                           p.d_model, err_word, stream);
     if (e != cudaSuccess) return e;
     if (p.T_new > 0) {
@@ -480,7 +495,7 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
     e = launch_dependent(ln_gate_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, stream, attn,
                          uvqk, 4 * F, gate, T, p.ln_eps);
     if (e != cudaSuccess) return e;
-    e = gemm_launch<EPI_RESIDUAL>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+    e = gemm_launch<EPI_RESIDUAL, 128>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
                                   err_word, stream);
     if (e != cudaSuccess) return e;
   }

@@ -89,6 +89,16 @@ def test_bf16_tcgen05_few_short_users(lengths):
     assert_bf16_close(got, ref, f"short users {lengths}", mag=case_magnitudes(case))
 
 
+def test_bf16_tcgen05_over_1024_users():
+    """1100 short users: the launch runs as chunks of at most 1024 users over
+    absolute rows (position + time bias)."""
+    rng = np.random.default_rng(15)
+    lengths = rng.integers(1, 40, size=1100)
+    case = workloads.jagged_case(15, lengths, H=2, d=128, dtype="bf16", n_pos=16, n_time=8)
+    got, ref = run_case(case)
+    assert_bf16_close(got, ref, "1100 users", mag=case_magnitudes(case))
+
+
 def test_bf16_tcgen05_pos_time_rab():
     case = workloads.jagged_case(8, [200, 640, 37, 1100], H=4, d=128, dtype="bf16", n_pos=128,
                                  n_time=64)
