@@ -45,6 +45,9 @@ struct AttnProblem {
   // callers without a workspace (hstu_attn_fwd, the uncached block) never
   // split keys over CTAs
   bool allow_split = true;
+  // launch with programmatic dependent launch (off for the uncached block
+  // stack, where the early-scheduled attention CTAs measured slower)
+  bool pdl = true;
 };
 
 // bf16, d == 128, tcgen05 path.  workspace: fp32 split partials (may be null if

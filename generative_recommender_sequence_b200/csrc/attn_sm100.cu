@@ -1443,12 +1443,13 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
-  cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq, tk,
-                                   tv, tkc, tvc, kp);
+  cudaError_t e = launch_kernel(p.pdl, kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq,
+                                tk, tv, tkc, tvc, kp);
   if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
   const int max_qt = std::max(1, (p.max_q + BM - 1) / BM);
-  return launch_dependent(split_reduce_kernel, dim3(BM / kReduceRows, (unsigned)(p.B * p.H * max_qt)),
-                          dim3(kReduceThreads), 0, stream, kp, max_qt);
+  return launch_kernel(p.pdl, split_reduce_kernel,
+                       dim3(BM / kReduceRows, (unsigned)(p.B * p.H * max_qt)), dim3(kReduceThreads), 0,
+                       stream, kp, max_qt);
 }
 
 // Key-split plan: one wave of (user, head, split) items, each streaming a long

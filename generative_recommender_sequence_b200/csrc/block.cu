@@ -16,14 +16,6 @@
 // accumulators (2 x BN columns), warps 2-9 drain the other accumulator
 // (tcgen05.ld -> epilogue -> global; two warps per TMEM lane quarter, BN/2
 // columns each) so the epilogue of tile i overlaps the main loop of tile i+1.
-//
-// Paired form (the wide projection): 2-CTA clusters own 256 x 256 tiles.
-// Each CTA loads its own 128 rows of A and 128 of the tile's 256 columns of
-// B, and CTA 0 issues tcgen05.mma.cta_group::2 (M=256, N=256) over both CTAs'
-// operands, each CTA receiving its 128 rows of the product in its own TMEM.
-// Per CTA that is 32 KiB of operands per 64-deep k-step instead of 48 KiB for
-// the same tensor work, which is what bounds the single-CTA 128 x 256 tile
-// (its operand stream from L2 is as fast as the tensor pipe consumes it).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,7 +25,6 @@
 
 #include "attn.h"
 #include "block.h"
-#include "pair.cuh"
 #include "sm100.cuh"
 
 namespace hstu {
@@ -48,26 +39,21 @@ constexpr int kBBoxBytes = GBK * 64 * 2;     // one 64-column B box: 8 KiB
 // Tile width BN (256 for the wide projection, 128 for the 512-column output
 // projection, whose 128 x 256 tiles would give 148 SMs only 1.4 waves) and the
 // TMA ring depth that keeps about 192 KiB of operands in flight.
-// PAIR: the tile is 256 x BN over a 2-CTA cluster and each CTA stages BN/2
-// columns of B.
-template <int BN, bool PAIR>
+template <int BN>
 struct GemmCfg {
-  static constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns staged per CTA
-  static constexpr int kBBytes = GBK * kBCols * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = kStageBytes >= 48 * 1024 ? 4 : 6;
+  static constexpr int kBBytes = GBK * BN * 2;
+  static constexpr int kStages = BN >= 256 ? 4 : 6;
   static constexpr int kEpiCols = BN / 2;    // columns per epilogue warp
-  static constexpr int kTileM = PAIR ? 2 * GBM : GBM;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN, true);
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(GBM, BN, true);
 };
 
 enum { EPI_SILU = 0, EPI_RESIDUAL = 1 };
 
-template <int BN, bool PAIR>
+template <int BN>
 struct __align__(1024) GemmSmem {
-  uint8_t a[GemmCfg<BN, PAIR>::kStages][kABytes];
-  uint8_t b[GemmCfg<BN, PAIR>::kStages][GemmCfg<BN, PAIR>::kBBytes];
-  uint64_t full[GemmCfg<BN, PAIR>::kStages], empty[GemmCfg<BN, PAIR>::kStages];
+  uint8_t a[GemmCfg<BN>::kStages][kABytes];
+  uint8_t b[GemmCfg<BN>::kStages][GemmCfg<BN>::kBBytes];
+  uint64_t full[GemmCfg<BN>::kStages], empty[GemmCfg<BN>::kStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -80,39 +66,25 @@ struct GemmParams {
   int* err;
 };
 
-// Commit helpers of the two forms: a single CTA's barrier, or the barrier at
-// the same offset in both CTAs of the pair.
-template <bool PAIR>
-__device__ __forceinline__ void gemm_commit(uint32_t bar) {
-  if (PAIR)
-    umma_commit_pair(bar);
-  else
-    umma_commit(bar);
-}
-
-template <int EPI, int BN, bool PAIR>
+template <int EPI, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b, const GemmParams P) {
-  using Cfg = GemmCfg<BN, PAIR>;
-  constexpr int GST = Cfg::kStages;
-  constexpr int kBCols = Cfg::kBCols;
-  constexpr int kEpiCols = Cfg::kEpiCols;
-  constexpr int kTileM = Cfg::kTileM;
-  // bytes the full barrier of a stage counts: both CTAs' halves in a pair
-  constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * Cfg::kStageBytes;
+  constexpr int GBN = BN;
+  constexpr int GST = GemmCfg<BN>::kStages;
+  constexpr int kBBytes = GemmCfg<BN>::kBBytes;
+  constexpr int kEpiCols = GemmCfg<BN>::kEpiCols;
+  constexpr uint32_t kIdescGemm = GemmCfg<BN>::kIdesc;
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem<BN, PAIR>& sm = *reinterpret_cast<GemmSmem<BN, PAIR>*>(
+  GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // rank in the pair; CTA 0 issues the MMAs and owns the full / acc_empty barriers
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   // dependent launch: barrier set-up and the TMEM allocation overlap the
-  // previous kernel's tail; global memory is touched only after the wait
-  pdl_launch_dependents();
-  const int m_tiles = (P.M + kTileM - 1) / kTileM, n_tiles = P.N / BN;
+  // previous kernel's tail; global memory is touched only after the wait.
+  // The next kernel is released only at the end (below): released at entry,
+  // its CTAs were scheduled onto SMs while this GEMM still ran, measured
+  // slower in the cached serving step.
+  const int m_tiles = (P.M + GBM - 1) / GBM, n_tiles = P.N / GBN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = P.K / GBK;
 
@@ -123,8 +95,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.acc_full[i]), 1);
-      // a pair's accumulator is drained by the epilogue warps of both CTAs
-      mbar_init(smem_u32(&sm.acc_empty[i]), (PAIR ? 2 : 1) * kEpiWarps);
+      mbar_init(smem_u32(&sm.acc_empty[i]), kEpiWarps);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
     fence_mbar_init();
@@ -132,19 +103,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tm_b);
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(smem_u32(&sm.tmem_base), 512);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(&sm.tmem_base), 512);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
   }
   pdl_wait();  // A (and, with the residual epilogue, the output) come from earlier kernels
   tc_fence_before();
   __syncthreads();
-  // the peer signals CTA 0's barriers only after both CTAs initialised theirs
-  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
@@ -152,59 +116,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       uint32_t c = 0;
       bool ok = true;
-      for (int t = unit; t < tiles && ok; t += units) {
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int mt = t / n_tiles, nt = t % n_tiles;
-        const int arow = mt * kTileM + (int)rank * GBM;
-        const int bcol = nt * BN + (int)rank * kBCols;
         for (int kb = 0; kb < kblocks; ++kb, ++c) {
           const uint32_t s = c % GST;
           if (!(ok = mbar_wait(smem_u32(&sm.empty[s]), ((c / GST) & 1) ^ 1))) break;
           const uint32_t bar = smem_u32(&sm.full[s]);
-          if (PAIR) {
-            // both CTAs' copies complete on CTA 0's barrier, which expects both
-            const uint32_t lbar = mapa_shared(bar, 0);
-            if (rank == 0) mbar_arrive_expect_tx(bar, kTxBytes);
-            tma_load_2d_pair(smem_u32(sm.a[s]), &tm_a, lbar, kb * GBK, arow);
+          mbar_arrive_expect_tx(bar, kABytes + kBBytes);
+          tma_load_2d(smem_u32(sm.a[s]), &tm_a, bar, kb * GBK, mt * GBM);
 #pragma unroll
-            for (int j = 0; j < kBCols / 64; ++j)
-              tma_load_2d_pair(smem_u32(sm.b[s]) + j * kBBoxBytes, &tm_b, lbar, bcol + j * 64,
-                               kb * GBK);
-          } else {
-            mbar_arrive_expect_tx(bar, kTxBytes);
-            tma_load_2d(smem_u32(sm.a[s]), &tm_a, bar, kb * GBK, arow);
-#pragma unroll
-            for (int j = 0; j < kBCols / 64; ++j)
-              tma_load_2d(smem_u32(sm.b[s]) + j * kBBoxBytes, &tm_b, bar, bcol + j * 64, kb * GBK);
-          }
+          for (int j = 0; j < GBN / 64; ++j)
+            tma_load_2d(smem_u32(sm.b[s]) + j * kBBoxBytes, &tm_b, bar, nt * GBN + j * 64, kb * GBK);
         }
       }
       if (!ok) {
         atomicExch(P.err, DEV_ERR_TIMEOUT);
-        if (PAIR && rank != 0) {
-          // this CTA's copies complete on CTA 0's barriers, which it cannot
-          // wait on: give any copy still in flight time to land before exit
-          const unsigned long long t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 200000ull) {
-          }
-        } else {
-          for (uint32_t i = 0; i < GST && i < c; ++i) {
-            const uint32_t cc = c - 1 - i;
-            mbar_wait(smem_u32(&sm.full[cc % GST]), (cc / GST) & 1);
-          }
+        for (uint32_t i = 0; i < GST && i < c; ++i) {
+          const uint32_t cc = c - 1 - i;
+          mbar_wait(smem_u32(&sm.full[cc % GST]), (cc / GST) & 1);
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // in a pair only CTA 0 issues (M = 256 MMAs over both CTAs' operands)
-    if (lane == 0 && rank == 0) {
+    if (lane == 0) {
       uint32_t c = 0, tcount = 0;
       bool ok = true;
-      for (int t = unit; t < tiles && ok; t += units, ++tcount) {
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
         const uint32_t ab = tcount & 1;
-        const uint32_t ebar = smem_u32(&sm.acc_empty[ab]);
-        const uint32_t epar = ((tcount >> 1) & 1) ^ 1;
-        if (!(ok = PAIR ? mbar_wait_cluster(ebar, epar) : mbar_wait(ebar, epar))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.acc_empty[ab]), ((tcount >> 1) & 1) ^ 1))) break;
         tc_fence_after();
         for (int kb = 0; kb < kblocks; ++kb, ++c) {
           const uint32_t s = c % GST;
@@ -215,22 +155,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < GBK / 16; ++kk) {
             const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
             // B is MN-major: 64-column boxes 8 KiB apart (LBO), 8-row k groups 1 KiB
-            // apart (SBO), 16 k-rows = 2 KiB per k-step (a pair's CTAs hold one
-            // column half each, in the same layout)
+            // apart (SBO), 16 k-rows = 2 KiB per k-step
             const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, kBBoxBytes, 1024);
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            if (PAIR)
-              umma_ss_pair(tmem + ab * BN, adesc, bdesc, Cfg::kIdesc, acc);
-            else
-              umma_ss(tmem + ab * BN, adesc, bdesc, Cfg::kIdesc, acc);
+            umma_ss(tmem + ab * GBN, adesc, bdesc, kIdescGemm, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          gemm_commit<PAIR>(smem_u32(&sm.empty[s]));
+          umma_commit(smem_u32(&sm.empty[s]));
         }
         if (!ok) break;
-        gemm_commit<PAIR>(smem_u32(&sm.acc_full[ab]));
+        umma_commit(smem_u32(&sm.acc_full[ab]));
       }
       if (!ok) atomicExch(P.err, DEV_ERR_TIMEOUT);
-      gemm_commit<PAIR>(smem_u32(&sm.mma_done));
+      umma_commit(smem_u32(&sm.mma_done));
       mbar_wait(smem_u32(&sm.mma_done), 0);
     }
     __syncwarp();
@@ -241,12 +176,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = sub * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     uint32_t tcount = 0;
-    for (int t = unit; t < tiles; t += units, ++tcount) {
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
       const int mt = t / n_tiles, nt = t % n_tiles;
       const uint32_t ab = tcount & 1;
-      const int64_t row = (int64_t)mt * kTileM + (int64_t)rank * GBM + r;
+      const int64_t row = (int64_t)mt * GBM + r;
       const bool valid = row < P.M;
-      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * BN + chalf * kEpiCols;
+      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN + chalf * kEpiCols;
       // residual epilogue: this thread's whole row segment of X is loaded
       // before the accumulator is ready (one memory latency per tile, hidden
       // behind the main loop, instead of one per 32-column chunk)
@@ -264,19 +199,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < kEpiCols / 32; ++ch) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_addr + ab * BN + chalf * kEpiCols + ch * 32, v);
+        tmem_ld32(tmem + lane_addr + ab * GBN + chalf * kEpiCols + ch * 32, v);
         tmem_wait_ld();
         reg_fence(v);
         if (ch == kEpiCols / 32 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            const uint32_t ebar = smem_u32(&sm.acc_empty[ab]);
-            if (PAIR && rank != 0)
-              mbar_arrive_cluster(mapa_shared(ebar, 0));
-            else
-              mbar_arrive(ebar);
-          }
+          if (lane == 0) mbar_arrive(smem_u32(&sm.acc_empty[ab]));
         }
         if (!valid) continue;
         float x[32];
@@ -313,17 +242,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   }
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
-  // neither CTA of a pair leaves (or frees tensor memory) while the other may
-  // still signal its barriers or read its operands
-  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR)
-      tmem_dealloc_pair(tmem, 512);
-    else
-      tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -379,16 +303,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-template <int BN, bool PAIR>
-size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, PAIR>) + 1024; }
+template <int BN>
+size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN>) + 1024; }
 
 // out[M, N] (ld ldo) = epi(A[M, K] (ld lda) @ B[K, N] (ld ldb)); residual
-// epilogue reads out before writing it.  PAIR runs 256 x GBN tiles on 2-CTA
-// clusters.
-template <int EPI, int GBN, bool PAIR>
+// epilogue reads out before writing it.
+template <int EPI, int GBN>
 cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb, void* out,
-                        int64_t ldo, int M, int N, int K, int* err, cudaStream_t stream) {
-  using Cfg = GemmCfg<GBN, PAIR>;
+                        int64_t ldo, int M, int N, int K, int* err, bool pdl, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   if (N % GBN != 0 || K % GBK != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
@@ -396,50 +318,21 @@ cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb,
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, Bw, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 2, 64, GBK))
     return cudaErrorInvalidValue;
-  auto kern = gemm_bf16_kernel<EPI, GBN, PAIR>;
-  const size_t smem = gemm_smem_bytes<GBN, PAIR>();
-  // per device: the shared-memory opt-in and, for pairs, how many 2-CTA
-  // clusters of this kernel can be resident at once
+  auto kern = gemm_bf16_kernel<EPI, GBN>;
   static bool attr_set[64] = {};
-  static int max_units[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  const bool cached = dev >= 0 && dev < 64 && attr_set[dev];
-  int units = cached ? max_units[dev] : 0;
-  if (!cached) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm_smem_bytes<GBN>());
     if (e != cudaSuccess) return e;
-    units = device_sm_count();
-    if (PAIR) {
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(2 * (units / 2));
-      cfg.blockDim = dim3(kGemmThreads);
-      cfg.dynamicSmemBytes = smem;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int clusters = 0;
-      e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-      if (e != cudaSuccess) return e;
-      if (clusters < 1) return cudaErrorInvalidConfiguration;
-      units = std::min(clusters, units / 2);
-    }
-    if (dev >= 0 && dev < 64) {
-      max_units[dev] = units;
-      attr_set[dev] = true;
-    }
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const int tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * (N / GBN);
-  const int grid_units = std::max(1, std::min(tiles, units));
+  const int tiles = ((M + GBM - 1) / GBM) * (N / GBN);
+  const int grid = std::max(1, std::min(tiles, device_sm_count()));
   GemmParams p{M, N, K, reinterpret_cast<__nv_bfloat16*>(out), ldo, err};
-  if (PAIR)
-    return launch_dependent_pairs(kern, dim3(2 * grid_units), dim3(kGemmThreads), smem, stream, ta,
-                                  tb, p);
-  return launch_dependent(kern, dim3(grid_units), dim3(kGemmThreads), smem, stream, ta, tb, p);
+  return launch_kernel(pdl, kern, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<GBN>(), stream, ta,
+                       tb, p);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -462,9 +355,14 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
   __nv_bfloat16* gate =
       reinterpret_cast<__nv_bfloat16*>(ws + align256((size_t)p.T * 4 * F * 2) + align256((size_t)p.T * F * 2));
   const int M = (int)p.T;
+  // The stack's kernels are launched stream-ordered, without programmatic
+  // dependent launch: with it, the attention CTAs scheduled early behind the
+  // projection GEMM cost 11-17 us per layer on B200 (8-layer stack 1223-1270
+  // vs 1132 us, same box).
+  constexpr bool kPdl = false;
   for (int l = 0; l < p.n_layers; ++l) {
-    cudaError_t e = gemm_launch<EPI_SILU, 256, true>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
-                                          p.d_model, err_word, stream);
+    cudaError_t e = gemm_launch<EPI_SILU, 256>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+                                          p.d_model, err_word, kPdl, stream);
     if (e != cudaSuccess) return e;
     AttnProblem a;
     a.B = p.B;
@@ -488,13 +386,14 @@ cudaError_t block_fwd_launch(const BlockProblem& p, void* workspace, size_t ws_b
     a.scale = p.scale;
     a.max_q = a.max_kv = p.max_len;
     a.allow_split = false;  // the block's workspace holds no split partials
+    a.pdl = kPdl;
     e = attn_sm100_launch(a, nullptr, 0, err_word, stream);
     if (e != cudaSuccess) return e;
-    e = launch_dependent(ln_gate_kernel, dim3((unsigned)((p.T + 7) / 8)), dim3(256), 0, stream,
-                         attn, uvqk, 4 * F, gate, p.T, p.ln_eps);
+    e = launch_kernel(kPdl, ln_gate_kernel, dim3((unsigned)((p.T + 7) / 8)), dim3(256), 0, stream,
+                      attn, uvqk, 4 * F, gate, p.T, p.ln_eps);
     if (e != cudaSuccess) return e;
-    e = gemm_launch<EPI_RESIDUAL, 128, false>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
-                                  err_word, stream);
+    e = gemm_launch<EPI_RESIDUAL, 128>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+                                  err_word, kPdl, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -581,8 +480,8 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
   for (int l = 0; l < p.n_layers; ++l) {
     const KvTableDev& t = p.tables[l];
     // [U | V | Q | K] = SiLU(X W1) for the new and the candidate rows at once
-    cudaError_t e = gemm_launch<EPI_SILU, 256, true>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
-                                          p.d_model, err_word, stream);
+    cudaError_t e = gemm_launch<EPI_SILU, 256>(p.x, p.d_model, p.w_uvqk[l], 4 * F, uvqk, 4 * F, M, 4 * F,
+                                          p.d_model, err_word, true, stream);
     if (e != cudaSuccess) return e;
     if (p.T_new > 0) {
       // the new tokens' K, V join this layer's cache, then they attend causally
@@ -605,8 +504,8 @@ cudaError_t block_cached_step_launch(const CachedStepProblem& p, void* workspace
     e = launch_dependent(ln_gate_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, stream, attn,
                          uvqk, 4 * F, gate, T, p.ln_eps);
     if (e != cudaSuccess) return e;
-    e = gemm_launch<EPI_RESIDUAL, 128, false>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
-                                  err_word, stream);
+    e = gemm_launch<EPI_RESIDUAL, 128>(gate, F, p.w_o[l], p.d_model, p.x, p.d_model, M, p.d_model, F,
+                                  err_word, true, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

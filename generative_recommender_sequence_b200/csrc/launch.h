@@ -9,16 +9,18 @@
 
 namespace hstu {
 
-// Launches `kernel` on `stream` with programmatic dependent launch enabled, so
-// its CTAs may be scheduled while the previous kernel of the stream finishes;
-// the kernel calls pdl_wait() before reading that kernel's results.
+// Launches `kernel` on `stream`; with `pdl` the launch carries programmatic
+// dependent launch, so its CTAs may be scheduled while the previous kernel of
+// the stream finishes (the kernel calls pdl_wait() before reading that
+// kernel's results).  Without it the launch is an ordinary stream-ordered one
+// and the kernel's pdl_wait() / pdl_launch_dependents() return at once.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                             cudaStream_t stream, Args&&... args) {
+cudaError_t launch_kernel(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
@@ -28,26 +30,11 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// The same with 2-CTA clusters along x (grid.x even): CTAs 2k and 2k + 1 form
-// one cluster.
+// The programmatic-dependent form, used by every kernel of the serving chain.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_dependent_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                   cudaStream_t stream, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 2;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+  return launch_kernel(true, kernel, grid, block, smem, stream, static_cast<Args&&>(args)...);
 }
 
 }  // namespace hstu
