@@ -16,6 +16,10 @@
 // accumulators (2 x BN columns), warps 2-9 drain the other accumulator
 // (tcgen05.ld -> epilogue -> global; two warps per TMEM lane quarter, BN/2
 // columns each) so the epilogue of tile i overlaps the main loop of tile i+1.
+// Each epilogue warp stages its 32 x 32 bf16 result boxes in shared memory
+// (two alternating 2 KiB buffers, 64-byte swizzle) and writes them with TMA
+// stores: a thread holds one row, so direct stores would touch 32 rows per
+// instruction (measured: 10 of GEMM1's 33 us went to those stores).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -49,10 +53,13 @@ struct GemmCfg {
 
 enum { EPI_SILU = 0, EPI_RESIDUAL = 1 };
 
+constexpr int kStageBoxBytes = 32 * 32 * 2;  // one 32 x 32 bf16 output box
+
 template <int BN>
 struct __align__(1024) GemmSmem {
   uint8_t a[GemmCfg<BN>::kStages][kABytes];
   uint8_t b[GemmCfg<BN>::kStages][GemmCfg<BN>::kBBytes];
+  uint8_t out[kEpiWarps][2][kStageBoxBytes];  // per epilogue warp, alternating
   uint64_t full[GemmCfg<BN>::kStages], empty[GemmCfg<BN>::kStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
@@ -66,10 +73,30 @@ struct GemmParams {
   int* err;
 };
 
+// TMA store of one shared-memory box to the tensor at (x, y), tracked as a
+// bulk group of the issuing thread.
+__device__ __forceinline__ void tma_store_2d(const void* desc, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(desc),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// until at most one of this thread's bulk groups still reads shared memory
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// until all of this thread's bulk groups have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// makes this thread's shared-memory writes visible to the TMA (async proxy)
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 template <int EPI, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_b, const GemmParams P) {
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_out, const GemmParams P) {
   constexpr int GBN = BN;
   constexpr int GST = GemmCfg<BN>::kStages;
   constexpr int kBBytes = GemmCfg<BN>::kBBytes;
@@ -101,6 +128,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -175,19 +203,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int chalf = (warp - 2) >> 2;
     const int r = sub * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+    uint8_t(&stage)[2][kStageBoxBytes] = sm.out[warp - 2];
+    // row `lane` of a 32 x 32 box: 64-byte rows, 16-byte chunk q stored at
+    // chunk q ^ ((row >> 1) & 3) (the TMA's 64-byte swizzle)
+    const int swz = (lane >> 1) & 3;
+    uint32_t ecount = 0;  // boxes this warp has staged
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
       const int mt = t / n_tiles, nt = t % n_tiles;
       const uint32_t ab = tcount & 1;
       const int64_t row = (int64_t)mt * GBM + r;
       const bool valid = row < P.M;
-      __nv_bfloat16* orow = P.out + row * P.ldo + (int64_t)nt * GBN + chalf * kEpiCols;
       // residual epilogue: this thread's whole row segment of X is loaded
       // before the accumulator is ready (one memory latency per tile, hidden
       // behind the main loop, instead of one per 32-column chunk)
       uint4 res[EPI == EPI_RESIDUAL ? kEpiCols / 8 : 1];
       if (EPI == EPI_RESIDUAL && valid) {
-        const uint4* src = reinterpret_cast<const uint4*>(orow);
+        const uint4* src = reinterpret_cast<const uint4*>(P.out + row * P.ldo + (int64_t)nt * GBN +
+                                                          chalf * kEpiCols);
 #pragma unroll
         for (int q = 0; q < kEpiCols / 8; ++q) res[q] = src[q];
       }
@@ -197,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < kEpiCols / 32; ++ch) {
+      for (int ch = 0; ch < kEpiCols / 32; ++ch, ++ecount) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_addr + ab * GBN + chalf * kEpiCols + ch * 32, v);
         tmem_wait_ld();
@@ -207,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.acc_empty[ab]));
         }
-        if (!valid) continue;
+        // rows past M are computed but not stored (the TMA store clips them)
         float x[32];
         if (EPI == EPI_SILU) {
 #pragma unroll
@@ -229,7 +262,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        uint8_t* buf = stage[ecount & 1];
+        // the store issued from this buffer two boxes ago must have read it
+        if (ecount >= 2) {
+          if (lane == 0) bulk_wait_read1();
+          __syncwarp();
+        }
+        uint4* srow = reinterpret_cast<uint4*>(buf + lane * 64);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 u;
@@ -237,10 +276,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           u.y = pack_bf16x2(x[q * 8 + 2], x[q * 8 + 3]);
           u.z = pack_bf16x2(x[q * 8 + 4], x[q * 8 + 5]);
           u.w = pack_bf16x2(x[q * 8 + 6], x[q * 8 + 7]);
-          dst[q] = u;
+          srow[q ^ swz] = u;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_out, smem_u32(buf), nt * GBN + chalf * kEpiCols + ch * 32,
+                       mt * GBM + sub * 32);
+          bulk_commit();
         }
       }
     }
+    // the output is complete (and the staging buffers free) before the CTA ends
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   pdl_launch_dependents();
   tc_fence_before();
@@ -318,6 +367,9 @@ cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb,
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, Bw, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 2, 64, GBK))
     return cudaErrorInvalidValue;
+  CUtensorMap to;
+  if (!make_tmap_2d_store(&to, out, (uint64_t)N, (uint64_t)M, (uint64_t)ldo * 2, 32, 32))
+    return cudaErrorInvalidValue;
   auto kern = gemm_bf16_kernel<EPI, GBN>;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -332,7 +384,7 @@ cudaError_t gemm_launch(const void* A, int64_t lda, const void* Bw, int64_t ldb,
   const int grid = std::max(1, std::min(tiles, device_sm_count()));
   GemmParams p{M, N, K, reinterpret_cast<__nv_bfloat16*>(out), ldo, err};
   return launch_kernel(pdl, kern, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<GBN>(), stream, ta,
-                       tb, p);
+                       tb, to, p);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
