@@ -77,6 +77,11 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
 
 constexpr int NTS = 4;              // key-timestamp ring depth
 constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
+// Round-balanced schedule of the contiguous causal launches (plan_rounds)
+constexpr int kRsMaxRounds = 32;   // items per CTA it can hold
+constexpr int kRsMaxLevels = 128;  // query tiles per user it can order
+constexpr int kRsMaxCtas = 160;    // grid size it can rank
+constexpr int kRsItemCost = 2;     // fixed cost of an item, in key tiles (fill + epilogue)
 constexpr int kRrowQuarters = 64;   // position-bias row per pointwise warp: 32 columns + 31
 constexpr int kRrowPairs = 96;      // same for the two-pair layout: 64 columns + 31
 constexpr int RROW = kRrowPairs;
@@ -121,6 +126,13 @@ struct __align__(1024) Smem {
   // balanced key splits: this CTA's one item (valid, user, query tile, head,
   // key-tile range), derived by plan_balanced
   int bal_ok, bal_b, bal_m, bal_h, bal_t0, bal_t1;
+  // round-balanced schedule (contiguous causal launches, plan_rounds): the
+  // number of rounds (0: the snake order applies), this CTA's item of each
+  // round, and the planner's per-CTA loads and per-level first item indices
+  int rs_rounds, rs_levels;
+  int rs_b[kRsMaxRounds], rs_m[kRsMaxRounds], rs_rem[kRsMaxRounds];
+  int rs_load[kRsMaxCtas];
+  int rs_first[kRsMaxLevels + 1];
 };
 
 struct KParams {
@@ -383,9 +395,122 @@ __device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
   if (blockIdx.x == 0 && lane == 0) P.plan[P.B] = base;
 }
 
-// The rnd-th item of this CTA: one fixed item with balanced splits (BAL),
-// otherwise the snake order over the longest-first item list.
-template <bool BAL>
+// Round-balanced schedule of a contiguous causal launch, planned identically
+// by every CTA (all threads call it).  The item list is the longest-first one
+// of Sched (query-tile level descending, then users, then heads); item t of
+// level m costs m + 1 key tiles plus kRsItemCost.  Round r hands items
+// [G r, G r + G) out in that order to the CTAs sorted by the load they already
+// carry (ties by CTA index), so the longest item of a round goes to the least
+// loaded CTA.  On C2/C4-like batches (a few hundred items of 1..26 tiles) this
+// bounds the busiest CTA close to the longest-processing-time rule, where the
+// snake order leaves it 13-15% above.  Batches with more rounds, levels or
+// CTAs than the tables hold keep the snake order (sm.rs_rounds = 0, items
+// decoded one at a time by decode_item).
+__device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x;
+  const int HS = H * n_split;
+  if (warp == 0) {
+    int mx = 0;
+    for (int b = lane; b < B; b += 32) mx = max(mx, q_tiles(sm.m_q, b, BM));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    bool ok = mx >= 1 && mx <= kRsMaxLevels && G <= kRsMaxCtas;
+    long long n = 0;
+    if (ok) {
+      // rs_first[k]: first item index of level mx - 1 - k
+      for (int k = 0; k < mx; ++k) {
+        if (lane == 0) sm.rs_first[k] = (int)n;
+        n += (long long)count_users_above(sm.m_q, B, mx - 1 - k, BM, lane) * HS;
+      }
+      if (lane == 0) sm.rs_first[mx] = (int)n;
+    }
+    const long long rounds = (n + G - 1) / G;
+    ok = ok && n > 0 && rounds <= kRsMaxRounds;
+    if (lane == 0) {
+      sm.rs_rounds = ok ? (int)rounds : 0;
+      sm.rs_levels = mx;
+    }
+  }
+  for (int c = tid; c < kRsMaxCtas; c += kThreads) sm.rs_load[c] = 0;
+  __syncthreads();
+  const int R = sm.rs_rounds;
+  if (R == 0) return;
+  const int mx = sm.rs_levels;  // rs_first[mx] is the item count
+  const int n_items = sm.rs_first[mx];
+  // four threads rank each CTA c: thread (c, part) compares against CTAs
+  // part, part + 4, ...; the counts are summed over the four lanes
+  const int c = tid >> 2, part = tid & 3;
+  for (int r = 0; r < R; ++r) {
+    int rank = 0;
+    if (c < G) {
+      const int key = sm.rs_load[c] * 256 + c;
+      for (int c2 = part; c2 < G; c2 += 4) rank += (sm.rs_load[c2] * 256 + c2) < key;
+    }
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+    __syncthreads();  // every rank is taken from the loads before this round
+    if (c < G && part == 0) {
+      const int t = r * G + rank;
+      int item = -1;
+      if (t < n_items) {
+        int k = 0;  // level index of item t: rs_first[k] <= t < rs_first[k + 1]
+        while (sm.rs_first[k + 1] <= t) ++k;
+        sm.rs_load[c] += (mx - k) + kRsItemCost;
+        item = t;
+      }
+      if (c == (int)blockIdx.x) sm.rs_b[r] = item;
+    }
+    __syncthreads();
+  }
+  // decode this CTA's items: level, user and head of item t
+  if (warp == 0) {
+    for (int r = 0; r < R; ++r) {
+      const int t = sm.rs_b[r];
+      int b = -1, m = 0, rem = 0;
+      if (t >= 0) {
+        int k = 0;
+        while (sm.rs_first[k + 1] <= t) ++k;
+        m = mx - 1 - k;
+        const int ri = t - sm.rs_first[k];
+        rem = ri % HS;
+        b = nth_user_above(sm.m_q, B, m, BM, ri / HS, lane);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        sm.rs_b[r] = b;
+        sm.rs_m[r] = m;
+        sm.rs_rem[r] = rem;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Item t of the longest-first list, decoded without state (walks the levels
+// from the top; warp-collective).  The round-balanced launches use it when
+// their batch does not fit plan_rounds' tables.
+__device__ __noinline__ bool decode_item(int B, int HS, const Smem& sm, long long t, int lane, int& b,
+                                         int& m, int& rem) {
+  long long base = 0;
+  for (int lvl = sm.rs_levels - 1; lvl >= 0; --lvl) {
+    const long long cnt = (long long)count_users_above(sm.m_q, B, lvl, BM, lane) * HS;
+    if (t < base + cnt) {
+      const long long r = t - base;
+      rem = (int)(r % HS);
+      b = nth_user_above(sm.m_q, B, lvl, BM, (int)(r / HS), lane);
+      m = lvl;
+      return b >= 0;
+    }
+    base += cnt;
+  }
+  return false;
+}
+
+// The rnd-th item of this CTA: one fixed item with balanced splits (BAL);
+// the round-balanced schedule of plan_rounds (RS); otherwise the snake order
+// over the longest-first item list.
+template <bool BAL, bool RS>
 __device__ __forceinline__ bool next_item(const KParams& P, const Smem& sm, Sched<BM>& sc,
                                           long long rnd, int lane, int& b, int& m, int& rem) {
   if (BAL) {
@@ -394,6 +519,16 @@ __device__ __forceinline__ bool next_item(const KParams& P, const Smem& sm, Sche
     m = sm.bal_m;
     rem = sm.bal_h;
     return true;
+  }
+  if (RS) {
+    if (sm.rs_rounds > 0) {
+      if (rnd >= sm.rs_rounds || sm.rs_b[rnd] < 0) return false;
+      b = sm.rs_b[rnd];
+      m = sm.rs_m[rnd];
+      rem = sm.rs_rem[rnd];
+      return true;
+    }
+    return decode_item(P.B, P.H * P.n_split, sm, snake_item(rnd), lane, b, m, rem);
   }
   return sc.item(snake_item(rnd), sm.m_q, lane, b, m, rem);
 }
@@ -521,6 +656,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
   const int tid = threadIdx.x;
+  // contiguous causal launches take the round-balanced schedule (plan_rounds)
+  constexpr bool RS = !PAGED && !CAND && !BAL;
   const int warp = tid >> 5, lane = tid & 31;
   // dependent launch: the next kernel may start being scheduled.  Barrier
   // initialisation, the descriptor prefetch and the TMEM allocation touch no
@@ -605,6 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.time_ext[i] = P.time_table ? P.time_table[min(i, P.n_time - 1)] : 0.f;
   }
   __syncthreads();
+  if (RS) plan_rounds(P.B, P.H, P.n_split, sm, tid);
   if (BAL && warp == 0) plan_balanced<CAND>(P, sm, lane);
   tc_fence_before();
   __syncthreads();
@@ -615,12 +753,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // =============================================== TMA producer
     Sched<BM> sc;
-    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
+    if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t kc = 0, vc = 0, qi = 0;
     bool ok = true;
     for (long long rnd = 0;; ++rnd) {
       int b, m, rem;
-      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       if (lane == 0) {
@@ -719,13 +857,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp 1 issues S = Q K^T, warp 3 issues O += P V.  Two issuers keep the
     // tensor pipe fed: while one waits on its barriers the other's MMAs run.
     Sched<BM> sc;
-    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
+    if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     const bool qk_role = warp == 1;
     uint32_t kc = 0, vc = 0, qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       const int nt = it.t1 - it.t0;
@@ -797,12 +935,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // time-gap bias, so the pointwise warps never wait on global loads.
     if (P.time_table != nullptr && !PAGED && !CAND) {
       Sched<BM> sc;
-      if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
+      if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
       uint32_t g = 0, qitem = 0;
       bool ok = true;
       for (long long rnd = 0; ok; ++rnd) {
         int b, m, rem;
-        if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+        if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
         const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
         if (it.t0 >= it.t1) continue;
         const long long base = it.n_k > 0 ? P.ts[it.kv_row0] : 0;
@@ -916,12 +1054,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pb_idx = -1;
     float pb_val = 0.f;
     Sched<BM> sc;
-    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
+    if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0, my_epi = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
@@ -1152,12 +1290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pb_idx = -1;
     float pb_val = 0.f;
     Sched<BM> sc;
-    if (!BAL) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
+    if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
-      if (!next_item<BAL>(P, sm, sc, rnd, lane, b, m, rem)) break;
+      if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
       // this row's query position (every candidate sits at the cached length)
@@ -1402,6 +1540,8 @@ __global__ void __launch_bounds__(kReduceThreads) split_reduce_kernel(KParams P,
 }
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
+// the 1 KiB alignment slack included: at most the 227 KiB a CTA may opt into
+static_assert(sizeof(Smem) + 1024 <= 232448, "attention shared memory exceeds the per-CTA limit");
 
 template <bool PAGED, bool CAND, bool PW2 = false, bool BAL = false>
 cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items, int num_sms,
