@@ -99,6 +99,22 @@ def test_bf16_tcgen05_over_1024_users():
     assert_bf16_close(got, ref, "1100 users", mag=case_magnitudes(case))
 
 
+@pytest.mark.parametrize("lengths,what", [
+    ([200] * 592, "32 rounds: the largest batch the round-balanced plan holds"),
+    ([200] * 593, "33 rounds: decoded item by item in the snake order"),
+    ([16500, 100, 3, 300], "129 query-tile levels: decoded item by item"),
+])
+def test_bf16_tcgen05_schedule_bounds(lengths, what):
+    """Contiguous causal launches plan a round-balanced item order in every
+    CTA when the batch fits the planner's tables (at most 32 rounds of the
+    SM count, 128 query-tile levels) and otherwise decode the snake order one
+    item at a time; both must cover every (user, head, query tile) once."""
+    case = workloads.jagged_case(16, lengths, H=4, d=128, dtype="bf16", n_pos=16, n_time=8)
+    rows = sample_rows(case.seq_offsets, 400)
+    got, ref = run_case(case, rows=rows)
+    assert_bf16_close(got, ref, what, mag=case_magnitudes(case, rows=rows))
+
+
 def test_bf16_tcgen05_pos_time_rab():
     case = workloads.jagged_case(8, [200, 640, 37, 1100], H=4, d=128, dtype="bf16", n_pos=128,
                                  n_time=64)
