@@ -401,9 +401,10 @@ __device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
 // level m costs m + 1 key tiles plus kRsItemCost.  Round r hands items
 // [G r, G r + G) out in that order to the CTAs sorted by the load they already
 // carry (ties by CTA index), so the longest item of a round goes to the least
-// loaded CTA.  On C2/C4-like batches (a few hundred items of 1..26 tiles) this
-// bounds the busiest CTA close to the longest-processing-time rule, where the
-// snake order leaves it 13-15% above.  Batches with more rounds, levels or
+// loaded CTA.  On jagged batches of a few hundred items of 1..26 tiles (8
+// users of 256..4096 tokens, 4 heads) this bounds the busiest CTA close to
+// the longest-processing-time rule, where the snake order leaves it 13-15%
+// above.  Batches with more rounds, levels or
 // CTAs than the tables hold keep the snake order (sm.rs_rounds = 0, items
 // decoded one at a time by decode_item).
 __device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, int tid) {
