@@ -68,6 +68,11 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid
                   uint64_t mid_stride_bytes, uint64_t outer_stride_bytes, uint32_t box_inner,
                   uint32_t box_outer);
 
+// 2-D bf16 tensor map [rows, inner] (row stride in bytes) for TMA stores of
+// box_rows x box_inner boxes staged in shared memory with the 64-byte swizzle.
+bool make_tmap_2d_store(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+
 int device_sm_count();
 
 }  // namespace hstu

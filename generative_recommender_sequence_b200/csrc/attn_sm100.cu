@@ -111,6 +111,9 @@ struct __align__(1024) Smem {
   TsSlot qts[2];               // query timestamps of the current / next item
   int pages[kPagesStaged];     // producer: page ids of the current item's key tiles
   uint64_t q_full[QST], q_empty[QST];
+  // q_done[s]: the 16 pointwise warps have finished with Q slot s after its
+  // item (output boxes staged there were read by their TMA stores)
+  uint64_t q_done[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   // s_full: one per buffer (16-warp layout) or per (pair, buffer) = tile mod 6
@@ -652,13 +655,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const __grid_constant__ CUtensorMap tm_kc,
-                           const __grid_constant__ CUtensorMap tm_vc, const KParams P) {
+                           const __grid_constant__ CUtensorMap tm_vc,
+                           const __grid_constant__ CUtensorMap tm_out, const KParams P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
   const int tid = threadIdx.x;
   // contiguous causal launches take the round-balanced schedule (plan_rounds)
   constexpr bool RS = !PAGED && !CAND && !BAL;
+  // ... and write their bf16 output through TMA stores staged in the finished
+  // item's Q slot
+  constexpr bool OST = RS;
   const int warp = tid >> 5, lane = tid & 31;
   // dependent launch: the next kernel may start being scheduled.  Barrier
   // initialisation, the descriptor prefetch and the TMEM allocation touch no
@@ -671,6 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < QST; ++i) {
       mbar_init(smem_u32(&sm.q_full[i]), 1);
       mbar_init(smem_u32(&sm.q_empty[i]), 1);
+      mbar_init(smem_u32(&sm.q_done[i]), 16);
     }
     for (int i = 0; i < KST; ++i) {
       mbar_init(smem_u32(&sm.k_full[i]), 1);
@@ -709,6 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_kc);
       tma_prefetch_desc(&tm_vc);
     }
+    if (OST) tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -765,6 +774,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const uint32_t qs = qi % QST;
         ok = mbar_wait(smem_u32(&sm.q_empty[qs]), ((qi / QST) & 1) ^ 1);
+        // the slot also holds the output boxes of the item two before
+        if (OST && ok && qi >= QST) ok = mbar_wait(smem_u32(&sm.q_done[qs]), ((qi / QST) - 1) & 1);
         if (ok) {
           const uint32_t bar = smem_u32(&sm.q_full[qs]);
           mbar_arrive_expect_tx(bar, kTileBytes);
@@ -1293,6 +1304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     Sched<BM> sc;
     if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0;
+    // an output box of the previous item still being read out of its Q slot
+    // by this warp's TMA store (released once the next item has begun)
+    bool box_pend = false;
+    uint32_t box_slot = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
@@ -1379,6 +1394,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait_warp(smem_u32(&sm.s_full[sb]), (g / NSP) & 1);
         if (!ok) break;
         tc_fence_after();
+        if (OST && box_pend) {
+          if (lane == 0) {
+            bulk_wait_read0();
+            mbar_arrive(smem_u32(&sm.q_done[box_slot]));
+          }
+          __syncwarp();
+          box_pend = false;
+        }
         // this warp's 32 S columns; its 16 P columns overwrite the first half
         // (chunk q of P goes to columns [8q, 8q + 8), already loaded as S)
         const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + cbase;
@@ -1434,7 +1457,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
-      if (row_ok) {
+      // a warp whose 32 rows all belong to the item writes its 32 x 32 box
+      // through the item's Q slot (no longer read: every MMA of the item is
+      // done) and one TMA store; per-thread row stores would touch 32 rows per
+      // instruction and stall the warp's next shared-memory reads behind them
+      const bool box_ok = OST && !P.partial && 32 * sub + 32 <= it.nvalid;
+      if (box_ok) {
+        uint8_t* buf = sm.q[qsl] + pwi * 2048;
+        const int swz = (lane >> 1) & 3;  // the TMA's 64-byte swizzle
+        uint4* srow = reinterpret_cast<uint4*>(buf + lane * 64);
+        const float sc2 = P.scale;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(oa[j]) * sc2, __uint_as_float(oa[j + 1]) * sc2);
+          u.y = pack_bf16x2(__uint_as_float(oa[j + 2]) * sc2, __uint_as_float(oa[j + 3]) * sc2);
+          u.z = pack_bf16x2(__uint_as_float(oa[j + 4]) * sc2, __uint_as_float(oa[j + 5]) * sc2);
+          u.w = pack_bf16x2(__uint_as_float(oa[j + 6]) * sc2, __uint_as_float(oa[j + 7]) * sc2);
+          srow[(j >> 3) ^ swz] = u;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_out, smem_u32(buf), it.h * HD + cbase, (int)(it.q_row0 + 32 * sub));
+          bulk_commit();
+        }
+        box_pend = true;
+        box_slot = qsl;
+      } else if (OST) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.q_done[qsl]));
+      }
+      if (row_ok && !box_ok) {
         if (P.partial) {
           // whole 32-byte sectors when the buffer allows: the scattered
           // per-row partial stores drain faster than as 16-byte pieces
@@ -1468,6 +1522,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++qi;
     }
     if (!ok && lane == 0) record_timeout(P, sm);
+    if (OST) {
+      // every output box is written before the CTA ends
+      if (lane == 0) {
+        bulk_wait_all();
+        if (box_pend) mbar_arrive(smem_u32(&sm.q_done[box_slot]));
+      }
+      __syncwarp();
+    }
   }
 
   // ---- teardown
@@ -1572,6 +1634,11 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     tvc = tq;
   }
   static_assert(PAGED || !BAL, "only paged launches split keys");
+  // contiguous causal launches store their bf16 output boxes with TMA
+  CUtensorMap tout = tq;
+  if (!PAGED && !CAND && !BAL && p.out != nullptr && !p.partial_only &&
+      !make_tmap_2d_store(&tout, p.out, (uint64_t)p.H * HD, qrows, (uint64_t)p.out_stride * 2, 32, 32))
+    return cudaErrorInvalidValue;
   auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PW2, BAL>;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -1585,7 +1652,7 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(items, num_sms));
   cudaError_t e = launch_kernel(p.pdl, kern, dim3(grid), dim3(kThreads), smem_bytes(), stream, tq,
-                                tk, tv, tkc, tvc, kp);
+                                tk, tv, tkc, tvc, tout, kp);
   if (e != cudaSuccess || kp.partial == nullptr || p.partial_only) return e;
   const int max_qt = std::max(1, (p.max_q + BM - 1) / BM);
   return launch_kernel(p.pdl, split_reduce_kernel,

@@ -3,7 +3,6 @@
 
 #include <cstddef>
 #include <cstdint>
-#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kv_table.h"
@@ -25,11 +24,6 @@ struct BlockProblem {
 };
 
 size_t block_workspace_bytes(int64_t T, int d_model, int H, int dh);
-
-// 2-D bf16 tensor map [rows, inner] (row stride in bytes) for TMA stores of
-// box_rows x box_inner boxes staged in shared memory with the 64-byte swizzle.
-bool make_tmap_2d_store(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
 
 // Largest user count of one cached step (the KV append grid's y extent).
 constexpr int kMaxCachedStepUsers = 65535;
