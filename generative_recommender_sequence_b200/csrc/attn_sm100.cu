@@ -663,9 +663,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x;
   // contiguous causal launches take the round-balanced schedule (plan_rounds)
   constexpr bool RS = !PAGED && !CAND && !BAL;
-  // ... and write their bf16 output through TMA stores staged in the finished
-  // item's Q slot
+  // Contiguous and paged causal launches write their bf16 output through TMA
+  // stores staged in the finished item's Q slot (16-warp and two-pair
+  // layouts respectively)
   constexpr bool OST = RS;
+  constexpr bool OST2 = PW2 && !CAND && !BAL;
   const int warp = tid >> 5, lane = tid & 31;
   // dependent launch: the next kernel may start being scheduled.  Barrier
   // initialisation, the descriptor prefetch and the TMEM allocation touch no
@@ -717,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_kc);
       tma_prefetch_desc(&tm_vc);
     }
-    if (OST) tma_prefetch_desc(&tm_out);
+    if (OST || OST2) tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -775,7 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t qs = qi % QST;
         ok = mbar_wait(smem_u32(&sm.q_empty[qs]), ((qi / QST) & 1) ^ 1);
         // the slot also holds the output boxes of the item two before
-        if (OST && ok && qi >= QST) ok = mbar_wait(smem_u32(&sm.q_done[qs]), ((qi / QST) - 1) & 1);
+        if ((OST || OST2) && ok && qi >= QST)
+          ok = mbar_wait(smem_u32(&sm.q_done[qs]), ((qi / QST) - 1) & 1);
         if (ok) {
           const uint32_t bar = smem_u32(&sm.q_full[qs]);
           mbar_arrive_expect_tx(bar, kTileBytes);
@@ -1068,12 +1071,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     Sched<BM> sc;
     if (!BAL && !RS) sc.init(sm.m_q, P.B, HS, lane);  // one fixed item per CTA otherwise
     uint32_t qi = 0, g = 0, my_epi = 0;
+    // an output box of this warp's last epilogue still being read out of its
+    // Q slot by a TMA store (released when the next item begins)
+    bool box_pend = false;
+    uint32_t box_slot = 0;
     bool ok = true;
     for (long long rnd = 0; ok; ++rnd) {
       int b, m, rem;
       if (!next_item<BAL, RS>(P, sm, sc, rnd, lane, b, m, rem)) break;
       const Item it = make_item<PAGED, CAND, BAL>(P, sm, b, m, rem);
       if (it.t0 >= it.t1) continue;
+      // release the previous item's Q slot here, not at this pair's next S
+      // tile: that tile may belong to the item after next, whose Q load waits
+      // for this release
+      if (OST2 && box_pend) {
+        if (lane == 0) {
+          bulk_wait_read0();
+          mbar_arrive(smem_u32(&sm.q_done[box_slot]));
+        }
+        __syncwarp();
+        box_pend = false;
+      }
       // this row's query position (every candidate sits at the cached length)
       const int64_t qp = CAND ? it.p0 : it.p0 + r;
       long long tq_i = 0;
@@ -1158,6 +1176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait_warp(smem_u32(&sm.s_full[g % (2 * NSP)]), (g / (2 * NSP)) & 1);
         if (!ok) break;
         tc_fence_after();
+
         // this warp's 64 S columns and, over their first half, its 32 P columns
         const uint32_t s_addr = tmem + lane_addr + TM_SP + sb * 128 + chalf * 64;
         const uint32_t p_addr = s_addr;
@@ -1221,6 +1240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the other pair can start the next item at once); this warp stores O
       // columns [64 chalf, 64 chalf + 64) of its 32 rows.
       if ((int)((g - 1) & 1) != wg) {
+        // this pair leaves the item's Q slot alone
+        if (OST2) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.q_done[qi & 1]));
+        }
         ++qi;
         continue;
       }
@@ -1232,6 +1256,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool row_ok = r < it.nvalid && it.q_row0 + r < P.total_q;
       const int64_t row = it.q_row0 + r;
+      // as in the 16-warp layout: whole 32-row boxes go through the item's Q
+      // slot (boxes 2 (pwi mod 8) + q of 2 KiB) and TMA stores
+      const bool box_ok = OST2 && !P.partial && 32 * sub + 32 <= it.nvalid;
+      const uint32_t qslot = qi & 1;
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
         const int ocol = 64 * chalf + 32 * q;
@@ -1243,6 +1271,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
+        }
+        if (box_ok) {
+          uint8_t* buf = sm.q[qslot] + ((pwi & 7) * 2 + q) * 2048;
+          const int swz = (lane >> 1) & 3;  // the TMA's 64-byte swizzle
+          uint4* srow = reinterpret_cast<uint4*>(buf + lane * 64);
+          const float sc2 = P.scale;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(oa[j]) * sc2, __uint_as_float(oa[j + 1]) * sc2);
+            u.y = pack_bf16x2(__uint_as_float(oa[j + 2]) * sc2, __uint_as_float(oa[j + 3]) * sc2);
+            u.z = pack_bf16x2(__uint_as_float(oa[j + 4]) * sc2, __uint_as_float(oa[j + 5]) * sc2);
+            u.w = pack_bf16x2(__uint_as_float(oa[j + 6]) * sc2, __uint_as_float(oa[j + 7]) * sc2);
+            srow[(j >> 3) ^ swz] = u;
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_out, smem_u32(buf), it.h * HD + ocol, (int)(it.q_row0 + 32 * sub));
+            bulk_commit();
+          }
+          continue;
         }
         if (!row_ok) continue;
         if (P.partial) {
@@ -1275,9 +1325,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (box_ok) {
+        box_pend = true;
+        box_slot = qslot;
+      } else if (OST2) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.q_done[qslot]));
+      }
       ++qi;
     }
     if (!ok && lane == 0) record_timeout(P, sm);
+    if (OST2) {
+      // every output box is written before the CTA ends
+      if (lane == 0) {
+        bulk_wait_all();
+        if (box_pend) mbar_arrive(smem_u32(&sm.q_done[box_slot]));
+      }
+      __syncwarp();
+    }
   } else if (warp >= 4) {
     // =============================================== pointwise + epilogue
     // 16 warps share every key tile: warp (cq, sub) takes score columns
@@ -1634,9 +1699,9 @@ cudaError_t launch_impl(const AttnProblem& p, const KParams& kp, long long items
     tvc = tq;
   }
   static_assert(PAGED || !BAL, "only paged launches split keys");
-  // contiguous causal launches store their bf16 output boxes with TMA
+  // causal launches without key splits store their bf16 output boxes with TMA
   CUtensorMap tout = tq;
-  if (!PAGED && !CAND && !BAL && p.out != nullptr && !p.partial_only &&
+  if (!CAND && !BAL && p.out != nullptr && !p.partial_only &&
       !make_tmap_2d_store(&tout, p.out, (uint64_t)p.H * HD, qrows, (uint64_t)p.out_stride * 2, 32, 32))
     return cudaErrorInvalidValue;
   auto kern = hstu_attn_sm100_kernel<PAGED, CAND, PW2, BAL>;
