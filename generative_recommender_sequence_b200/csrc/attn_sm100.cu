@@ -419,10 +419,11 @@ __device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, in
     for (int b = lane; b < B; b += 32) mx = max(mx, q_tiles(sm.m_q, b, BM));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    bool ok = mx >= 1 && mx <= kRsMaxLevels && G <= kRsMaxCtas;
+    // rs_first[k]: first item index of level mx - 1 - k (also what decode_item
+    // searches when the rounds do not fit)
+    const bool levels_ok = mx >= 1 && mx <= kRsMaxLevels;
     long long n = 0;
-    if (ok) {
-      // rs_first[k]: first item index of level mx - 1 - k
+    if (levels_ok) {
       for (int k = 0; k < mx; ++k) {
         if (lane == 0) sm.rs_first[k] = (int)n;
         n += (long long)count_users_above(sm.m_q, B, mx - 1 - k, BM, lane) * HS;
@@ -430,7 +431,7 @@ __device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, in
       if (lane == 0) sm.rs_first[mx] = (int)n;
     }
     const long long rounds = (n + G - 1) / G;
-    ok = ok && n > 0 && rounds <= kRsMaxRounds;
+    const bool ok = levels_ok && G <= kRsMaxCtas && n > 0 && rounds <= kRsMaxRounds;
     if (lane == 0) {
       sm.rs_rounds = ok ? (int)rounds : 0;
       sm.rs_levels = mx;
@@ -491,13 +492,29 @@ __device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, in
   }
 }
 
-// Item t of the longest-first list, decoded without state (walks the levels
-// from the top; warp-collective).  The round-balanced launches use it when
-// their batch does not fit plan_rounds' tables.
+// Item t of the longest-first list, decoded without state (warp-collective).
+// The round-balanced launches use it when their batch does not fit
+// plan_rounds' round tables: with at most kRsMaxLevels levels the per-level
+// first items are in rs_first (binary search), otherwise the levels are
+// walked from the top.
 __device__ __noinline__ bool decode_item(int B, int HS, const Smem& sm, long long t, int lane, int& b,
                                          int& m, int& rem) {
+  const int mx = sm.rs_levels;
+  if (mx >= 1 && mx <= kRsMaxLevels) {
+    if (t >= sm.rs_first[mx]) return false;
+    int lo = 0, hi = mx - 1;  // largest k with rs_first[k] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.rs_first[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int r = (int)(t - sm.rs_first[lo]);
+    rem = r % HS;
+    m = mx - 1 - lo;
+    b = nth_user_above(sm.m_q, B, m, BM, r / HS, lane);
+    return b >= 0;
+  }
   long long base = 0;
-  for (int lvl = sm.rs_levels - 1; lvl >= 0; --lvl) {
+  for (int lvl = mx - 1; lvl >= 0; --lvl) {
     const long long cnt = (long long)count_users_above(sm.m_q, B, lvl, BM, lane) * HS;
     if (t < base + cnt) {
       const long long r = t - base;
