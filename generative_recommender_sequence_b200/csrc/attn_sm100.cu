@@ -78,7 +78,10 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
 constexpr int NTS = 4;              // key-timestamp ring depth
 constexpr int kPagesStaged = 512;  // page ids staged per item (128 key tiles)
 // Round-balanced schedule of the contiguous causal launches (plan_rounds)
-constexpr int kRsMaxRounds = 32;   // items per CTA it can hold
+// items per CTA it plans: short-sequence batches (a few hundred items, 3
+// rounds) gain from it, long ones (17 rounds, users of up to 128 query tiles)
+// ran 6.5% slower than in the snake order, which they keep
+constexpr int kRsMaxRounds = 8;
 constexpr int kRsMaxLevels = 128;  // query tiles per user it can order
 constexpr int kRsMaxCtas = 160;    // grid size it can rank
 constexpr int kRsItemCost = 2;     // fixed cost of an item, in key tiles (fill + epilogue)
@@ -407,9 +410,9 @@ __device__ void plan_balanced(const KParams& P, Smem& sm, int lane) {
 // loaded CTA.  On jagged batches of a few hundred items of 1..26 tiles (8
 // users of 256..4096 tokens, 4 heads) this bounds the busiest CTA close to
 // the longest-processing-time rule, where the snake order leaves it 13-15%
-// above.  Batches with more rounds, levels or
-// CTAs than the tables hold keep the snake order (sm.rs_rounds = 0, items
-// decoded one at a time by decode_item).
+// above.  Batches with more rounds (long sequences: there the snake order
+// measured faster), levels or CTAs than the tables hold keep the snake order
+// (sm.rs_rounds = 0, items decoded one at a time by decode_item).
 __device__ __noinline__ void plan_rounds(int B, int H, int n_split, Smem& sm, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;

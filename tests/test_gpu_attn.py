@@ -100,14 +100,14 @@ def test_bf16_tcgen05_over_1024_users():
 
 
 @pytest.mark.parametrize("lengths,what", [
-    ([200] * 592, "32 rounds: the largest batch the round-balanced plan holds"),
-    ([200] * 593, "33 rounds: decoded item by item in the snake order"),
+    ([200] * 148, "8 rounds: the largest batch the round-balanced plan takes"),
+    ([200] * 149, "9 rounds: decoded item by item in the snake order"),
     ([16500, 100, 3, 300], "129 query-tile levels: decoded item by item"),
 ])
 def test_bf16_tcgen05_schedule_bounds(lengths, what):
     """Contiguous causal launches plan a round-balanced item order in every
-    CTA when the batch fits the planner's tables (at most 32 rounds of the
-    SM count, 128 query-tile levels) and otherwise decode the snake order one
+    CTA when the batch fits the planner's tables (at most 8 rounds of the SM
+    count, 128 query-tile levels) and otherwise decode the snake order one
     item at a time; both must cover every (user, head, query tile) once."""
     case = workloads.jagged_case(16, lengths, H=4, d=128, dtype="bf16", n_pos=16, n_time=8)
     rows = sample_rows(case.seq_offsets, 400)
