@@ -21,16 +21,20 @@
 //   warp 3      tcgen05 issuer of O += P V, P read from TMEM (bf16 P written over
 //               the start of each warpgroup's S columns)
 //   warp 2      stages key timestamps for the time-gap bias (mbarrier ring)
-//   warps 4-19  four "pointwise" warpgroups: two pairs alternate key tiles, the
-//               two warpgroups of a pair split the tile's 128 score columns;
-//               read S from TMEM, add the biases, mask, SiLU (via tanh), pack
-//               P to bf16 in TMEM; the pair that took an item's last key tile
-//               also runs its epilogue (O * scale -> bf16 or fp32 split partial)
-//               while the other pair starts the next item.
+//   warps 4-19  16 "pointwise" warps: read S from TMEM, add the biases, mask,
+//               SiLU (via tanh), pack P to bf16 in TMEM, then run the item's
+//               epilogue (O * scale -> bf16, or the fp32 partial of a key
+//               split).  Paged causal launches split them into two pairs that
+//               alternate key tiles (the pair that took an item's last tile runs
+//               its epilogue while the other starts the next item); the other
+//               launches share every tile among all 16.  Causal launches without
+//               key splits stage whole 32 x 32 output boxes in the finished
+//               item's Q slot and write them with TMA stores.
 // There is no softmax, so there is no running max and no rescaling of O, and
 // key splits of one query tile add exactly (the candidate path splits keys).
 // Work items (user, head, query tile, split) run longest-first: query tiles
-// are visited from the highest tile index down.
+// are visited from the highest tile index down, handed to the CTAs in a snake
+// order, or (short contiguous causal batches) by the round-balanced plan.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
