@@ -19,7 +19,9 @@
 // Each epilogue warp stages its 32 x 32 bf16 result boxes in shared memory
 // (two alternating 2 KiB buffers, 64-byte swizzle) and writes them with TMA
 // stores: a thread holds one row, so direct stores would touch 32 rows per
-// instruction (measured: 10 of GEMM1's 33 us went to those stores).
+// instruction (measured: 10 of GEMM1's 33 us went to those stores).  The
+// residual epilogue TMA-loads the tile's X boxes into the same two buffers
+// while the main loop runs, adds them there and stores the sums back.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -62,6 +64,7 @@ struct __align__(1024) GemmSmem {
   uint8_t out[kEpiWarps][2][kStageBoxBytes];  // per epilogue warp, alternating
   uint64_t full[GemmCfg<BN>::kStages], empty[GemmCfg<BN>::kStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t x_full[kEpiWarps];  // residual epilogue: X boxes of the tile landed
   uint64_t mma_done;
   uint32_t tmem_base;
 };
@@ -106,6 +109,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(smem_u32(&sm.acc_empty[i]), kEpiWarps);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
+    for (int i = 0; i < kEpiWarps; ++i) mbar_init(smem_u32(&sm.x_full[i]), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
@@ -182,7 +186,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // epilogue warps 2..9: TMEM lane quarter = warp % 4, column half by warp
     const int sub = warp & 3;
     const int chalf = (warp - 2) >> 2;
-    const int r = sub * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
     uint8_t(&stage)[2][kStageBoxBytes] = sm.out[warp - 2];
     // row `lane` of a 32 x 32 box: 64-byte rows, 16-byte chunk q stored at
@@ -193,19 +196,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
       const int mt = t / n_tiles, nt = t % n_tiles;
       const uint32_t ab = tcount & 1;
-      const int64_t row = (int64_t)mt * GBM + r;
-      const bool valid = row < P.M;
-      // residual epilogue: this thread's whole row segment of X is loaded
-      // before the accumulator is ready (one memory latency per tile, hidden
-      // behind the main loop, instead of one per 32-column chunk)
-      uint4 res[EPI == EPI_RESIDUAL ? kEpiCols / 8 : 1];
-      if (EPI == EPI_RESIDUAL && valid) {
-        const uint4* src = reinterpret_cast<const uint4*>(P.out + row * P.ldo + (int64_t)nt * GBN +
-                                                          chalf * kEpiCols);
+      // residual epilogue (kEpiCols = 64: two boxes per warp, one per staging
+      // buffer): the tile's X boxes are TMA-loaded into the buffers before the
+      // accumulator is ready, once the previous tile's stores have read them
+      static_assert(EPI != EPI_RESIDUAL || kEpiCols == 64, "residual epilogue stages two boxes");
+      if (EPI == EPI_RESIDUAL) {
+        if (lane == 0) {
+          bulk_wait_read0();
+          const uint32_t xb = smem_u32(&sm.x_full[warp - 2]);
+          mbar_arrive_expect_tx(xb, 2 * kStageBoxBytes);
 #pragma unroll
-        for (int q = 0; q < kEpiCols / 8; ++q) res[q] = src[q];
+          for (int ch = 0; ch < 2; ++ch)
+            tma_load_2d(smem_u32(stage[ch]), &tm_out, xb, nt * GBN + chalf * kEpiCols + ch * 32,
+                        mt * GBM + sub * 32);
+        }
+        __syncwarp();
       }
-      if (!mbar_wait_warp(smem_u32(&sm.acc_full[ab]), (tcount >> 1) & 1)) {
+      if (!mbar_wait_warp(smem_u32(&sm.acc_full[ab]), (tcount >> 1) & 1) ||
+          (EPI == EPI_RESIDUAL && !mbar_wait_warp(smem_u32(&sm.x_full[warp - 2]), tcount & 1))) {
         if (lane == 0) atomicExch(P.err, DEV_ERR_TIMEOUT);
         break;
       }
@@ -231,9 +239,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             x[j] = fmaf(h, tanh_approx(h), h);
           }
         } else {
+          const uint4* xrow = reinterpret_cast<const uint4*>(stage[ch] + lane * 64);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint4 u = res[EPI == EPI_RESIDUAL ? ch * 4 + q : 0];
+            const uint4 u = xrow[q ^ swz];
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -243,9 +252,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        uint8_t* buf = stage[ecount & 1];
+        uint8_t* buf = stage[EPI == EPI_RESIDUAL ? ch : (ecount & 1)];
         // the store issued from this buffer two boxes ago must have read it
-        if (ecount >= 2) {
+        if (EPI != EPI_RESIDUAL && ecount >= 2) {
           if (lane == 0) bulk_wait_read1();
           __syncwarp();
         }
