@@ -177,6 +177,20 @@ def test_causal_suffix_query_blocks(lengths):
     table.close()
 
 
+def test_causal_suffix_many_single_tile_items():
+    """Mostly one-tile users between longer ones: in the two-pair layout the pair
+    that writes an item's output boxes through its Q slot often takes its next
+    tile from the item after next, whose Q load waits for that slot."""
+    lengths = [1, 64, 128, 5, 700, 30, 127, 3, 128, 17, 260, 2, 90, 128, 33, 1]
+    case = workloads.long_history(lengths=lengths, pool_tokens=8192)
+    table = make_table(case)
+    users = dev(case.users)
+    prefill(table, case, users)
+    out = step(table, case, users)
+    assert_bf16_close(to_np(out), oracle_out(case), "single-tile items", mag=oracle_mag(case))
+    table.close()
+
+
 def test_causal_suffix_long_runs_behind_history():
     """Query suffixes of 256-700 rows after long cached histories (tile rows start
     past position 0)."""
