@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kCopyThreads)
 // Every CTA reads the listed users' lengths and page counts and the free-stack
 // top at entry and re-derives the whole batch's allocation from them
 // (validation, per-user page demand, exclusive scan in listed order, pages
-// popped from the top of the stack), so all CTAs reach the same verdict and
+// popped from the top of the stack), so all CTAs reach the same decision and
 // the same page ids without waiting on each other.  CTA (c, b) copies tokens
 // [2c, 2c + 2) of user b into their slots; CTA (0, b) also writes user b's new
 // page-list entries and its lookup row.  None of the state read at entry is
@@ -575,7 +575,7 @@ __global__ void __launch_bounds__(kCopyThreads)
       }
     }
   }
-  if (!ok) return;  // the same verdict in every CTA (every thread of it)
+  if (!ok) return;  // the same decision in every CTA (every thread of it)
   __syncthreads();
   if (PLAN) {
     if (tid == 0) {

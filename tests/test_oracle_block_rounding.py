@@ -56,16 +56,16 @@ def _from_pieces(c, round_output=True):
     """One layer from separately pinned pieces, rounded where the GPU stores bf16."""
     x, T = c["x"], c["x"].shape[0]
     z = torch.from_numpy(x) @ torch.from_numpy(c["w1"][0])                    # fp64 matmul
-    uvqk = _bf(torch.nn.functional.silu(z).numpy())                          # round 1
+    uvqk = _bf(torch.nn.functional.silu(z).numpy())                          # rounding point 1
     U, V, Q, K = (uvqk[:, i * F:(i + 1) * F] for i in range(4))
     a = oracle.attn_causal(Q.reshape(T, H, DH), K.reshape(T, H, DH), V.reshape(T, H, DH), c["off"],
                            timestamps=c["ts"], pos_table=c["pos"], time_table=c["tim"],
                            scale=c["scale"]).reshape(T, F)
-    A = _bf(a)                                                               # round 2
+    A = _bf(a)                                                               # rounding point 2
     ln = torch.nn.functional.layer_norm(torch.from_numpy(A), (F,), eps=EPS).numpy()
-    G = _bf(ln * U)                                                          # round 3
+    G = _bf(ln * U)                                                          # rounding point 3
     y = x + (torch.from_numpy(G) @ torch.from_numpy(c["w2"][0])).numpy()
-    return _bf(y) if round_output else y                                     # round 4
+    return _bf(y) if round_output else y                                     # rounding point 4
 
 
 def _oracle_layer(c, fn=None, round_output=True):
